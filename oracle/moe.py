@@ -1,0 +1,98 @@
+"""Routed MoE layer forward oracle over 4-bit expert stacks (test infrastructure only).
+
+Sources on the pages:
+
+* "MoE Training & Inference Guides", ``grouped-nf4-gemm`` table: the routed MoE
+  expert GEMM runs straight on NF4 packed weights (``gemm_4bit_grouped``) or on
+  the released E2M1 blocks and E8M0 scales (``gemm_mxfp4_grouped``), with fp32
+  accumulation and no bf16 expert tensor; and ``ExpertsLoRA`` adds a per-expert
+  low-rank delta before each routed expert's activation.
+* "experts4bit-qlora" package page, limits list: the fast engines assume the
+  stock expert epilogue act(gate) * up, with no biases or clamps
+  (``EpilogueContractError`` otherwise).
+* "experts4bit-qlora" package page, "What it does": the experts of a layer are
+  one fused three-dimensional parameter ``[E, ...]``.
+* Examples on the pages use LoRA rank r = 8 and alpha = 16.
+
+The forward, in the pages' order and with every product in fp64:
+
+1. route: ids and gate weights per token (:mod:`oracle.route`);
+2. permute: routed rows grouped by expert, stable in slot order;
+3. per expert e, on its rows X_e: G = X_e W_gu[e] (+ s * (X_e A_e) B_e with
+   s = alpha / r); h = silu(G[:, :I]) * G[:, I:], silu(z) = z / (1 + e^-z);
+   Y_e = h W_dn[e];
+4. combine: out[t] = sum_j w[t, j] * y[slot (t, j)], j ascending.
+
+Readings where the pages are silent:
+
+* Logical shapes gate_up [E, H, 2I] and down [E, I, H]; each expert's matrix is
+  STORED transposed and K-contiguous, gate_up as [2I, H] and down as [H, I],
+  so quantisation blocks run along the reduction dimension (the MX layout and
+  the released gpt-oss blocks layout).
+* The fused 2I output is [gate | up] halves, not interleaved (interleaving is
+  named on the MXFP4 page as a gpt-oss peculiarity, outside the stock epilogue).
+* One LoRA adapter per expert on the fused gate_up output: A_e [H, r],
+  B_e [r, 2I].
+"""
+import numpy as np
+
+from .bf16 import bf16_bits_to_f64
+from .mxfp4 import decode_mxfp4
+from .nf4 import decode_nf4
+from .route import route
+
+NF4 = "nf4"
+MXFP4 = "mxfp4"
+
+
+def decode_expert(fmt, codes, scales, e, rows, cols):
+    """fp64 matrix [rows, cols] of expert e from a flat stored stack [E, rows, cols]."""
+    per = rows * cols
+    c = np.asarray(codes).reshape(-1)[e * per // 2:(e + 1) * per // 2]
+    if fmt == NF4:
+        s = np.asarray(scales).reshape(-1)[e * per // 64:(e + 1) * per // 64]
+        return decode_nf4(c, s, per).reshape(rows, cols)
+    if fmt == MXFP4:
+        s = np.asarray(scales).reshape(-1)[e * per // 32:(e + 1) * per // 32]
+        return decode_mxfp4(c, s, per).reshape(rows, cols)
+    raise ValueError(fmt)
+
+
+def silu(z):
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def moe_forward(x_bits, logits_bits, k, fmt, E, H, I, gu_codes, gu_scales, dn_codes, dn_scales,
+                lora_A_bits=None, lora_B_bits=None, lora_scale=0.0):
+    """Layer forward.  x: bf16 bits [T, H]; logits: bf16 bits [T, E].  Returns (out fp64 [T, H], route dict)."""
+    x = bf16_bits_to_f64(np.asarray(x_bits, dtype=np.uint16)).reshape(-1, H)
+    T = x.shape[0]
+    r = route(np.asarray(logits_bits, dtype=np.uint16).reshape(T, E), k)
+    offsets, sorted_slot = r["offsets"], r["sorted_slot"]
+    x_sorted = x[sorted_slot // k]                       # step 2: permute
+    y_sorted = np.zeros((T * k, H), dtype=np.float64)
+    lora = lora_A_bits is not None
+    if lora:
+        A = bf16_bits_to_f64(np.asarray(lora_A_bits, dtype=np.uint16))
+        B = bf16_bits_to_f64(np.asarray(lora_B_bits, dtype=np.uint16))
+        rank = A.size // (E * H)
+        A = A.reshape(E, H, rank)
+        B = B.reshape(E, rank, 2 * I)
+    for e in range(E):                                   # step 3: per expert
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if lo == hi:
+            continue
+        Xe = x_sorted[lo:hi]
+        Wgu = decode_expert(fmt, gu_codes, gu_scales, e, 2 * I, H)     # [2I, H]
+        G = Xe @ Wgu.T
+        if lora:
+            G = G + lora_scale * ((Xe @ A[e]) @ B[e])
+        h = silu(G[:, :I]) * G[:, I:]
+        Wdn = decode_expert(fmt, dn_codes, dn_scales, e, H, I)         # [H, I]
+        y_sorted[lo:hi] = h @ Wdn.T
+    out = np.zeros((T, H), dtype=np.float64)             # step 4: combine, j ascending
+    for j in range(k):
+        pos = r["slot_pos"][np.arange(T) * k + j]
+        out += r["w64"][:, j:j + 1] * y_sorted[pos]
+    return out, r

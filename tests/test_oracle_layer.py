@@ -1,0 +1,172 @@
+"""Pins for the routing and layer-forward oracles.
+
+Routing is checked against a per-token brute-force sort; the grouped forward
+against a per-token dense loop written independently here, against the
+textbook dense SwiGLU FFN (E = 1, k = 1), against token permutation and
+against a zero LoRA B.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from bit_mixture_experts_top_b200 import synth
+from oracle import bf16, moe, mxfp4, nf4, route
+
+
+def _brute_topk(row, k):
+    return [e for _, e in sorted(((-v, e) for e, v in enumerate(row)))][:k]
+
+
+@pytest.mark.parametrize("T,E,k", [(50, 8, 2), (40, 128, 8), (7, 32, 4), (3, 5, 5)])
+def test_route_matches_brute_force(T, E, k):
+    g = np.random.default_rng(T * E + k)
+    # few distinct values -> many ties; include -0.0 and +0.0
+    vals = np.array([-1.0, -0.0, 0.0, 0.5, 0.5, 2.0], np.float32)
+    logits = synth.to_bf16_bits(g.choice(vals, size=(T, E)))
+    r = route.route(logits, k)
+    lf = bf16.bf16_bits_to_f64(logits)
+    for t in range(T):
+        assert list(r["ids"][t]) == _brute_topk(lf[t], k)
+
+
+def test_route_constant_rows_take_lowest_ids():
+    logits = synth.to_bf16_bits(np.full((4, 16), 1.25, np.float32))
+    r = route.route(logits, 3)
+    assert np.array_equal(r["ids"], np.tile([0, 1, 2], (4, 1)))
+    assert np.allclose(r["w64"], 1.0 / 3.0, rtol=0, atol=1e-15)
+
+
+def test_route_weights_equal_renormalised_full_softmax():
+    g = np.random.default_rng(5)
+    logits = synth.to_bf16_bits(g.standard_normal((64, 32)))
+    r = route.route(logits, 4)
+    lf = bf16.bf16_bits_to_f64(logits)
+    full = np.exp(lf) / np.exp(lf).sum(axis=1, keepdims=True)
+    sel = np.take_along_axis(full, r["ids"].astype(np.int64), axis=1)
+    assert np.allclose(r["w64"], sel / sel.sum(axis=1, keepdims=True), rtol=1e-13, atol=0)
+    assert np.all(np.diff(r["w64"], axis=1) <= 0)          # ordered by logit
+
+
+def test_route_permutation_is_stable_grouping():
+    g = np.random.default_rng(6)
+    T, E, k = 300, 16, 3
+    r = route.route(synth.to_bf16_bits(g.standard_normal((T, E))), k)
+    ids = r["ids"].reshape(-1)
+    ss, off = r["sorted_slot"], r["offsets"]
+    assert sorted(ss.tolist()) == list(range(T * k))
+    assert off[0] == 0 and off[-1] == T * k
+    for e in range(E):
+        grp = ss[off[e]:off[e + 1]]
+        assert np.all(ids[grp] == e) and np.all(np.diff(grp) > 0)
+        assert r["counts"][e] == grp.size
+    assert np.array_equal(ss[r["slot_pos"]], np.arange(T * k))
+
+
+# ---------------------------------------------------------------- layer forward
+
+def _tiny_layer(fmt, E, H, I, seed=0):
+    if fmt == "mxfp4":
+        gu = synth.stack_mxfp4(E, 2 * I, H, -4, 2, seed, "gu")
+        dn = synth.stack_mxfp4(E, H, I, -4, 2, seed, "dn")
+    else:
+        gu = nf4.quantize_nf4(synth.stack_normal_f32(E, 2 * I, H, 0.02, seed, "gu"))
+        dn = nf4.quantize_nf4(synth.stack_normal_f32(E, H, I, 0.02, seed, "dn"))
+    return gu, dn
+
+
+def _decode(fmt, codes, scales, e, rows, cols):
+    per = rows * cols
+    c = codes[e * per // 2:(e + 1) * per // 2]
+    if fmt == "mxfp4":
+        return mxfp4.decode_mxfp4(c, scales[e * per // 32:(e + 1) * per // 32], per).reshape(rows, cols)
+    return nf4.decode_nf4(c, scales[e * per // 64:(e + 1) * per // 64], per).reshape(rows, cols)
+
+
+def _dense_loop(fmt, x, logits, k, E, H, I, gu, dn, A=None, B=None, s=0.0):
+    """Per token, per choice: decode the chosen expert and apply it to that token alone."""
+    xf = bf16.bf16_bits_to_f64(x)
+    lf = bf16.bf16_bits_to_f64(logits)
+    out = np.zeros((xf.shape[0], H))
+    for t in range(xf.shape[0]):
+        ids = _brute_topk(lf[t], k)
+        z = np.array([lf[t, e] for e in ids])
+        w = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+        for j, e in enumerate(ids):
+            wgu = _decode(fmt, gu[0], gu[1], e, 2 * I, H)
+            wdn = _decode(fmt, dn[0], dn[1], e, H, I)
+            g = np.array([sum(xf[t, c] * wgu[n, c] for c in range(H)) for n in range(2 * I)]) \
+                if H * I <= 64 * 32 else wgu @ xf[t]
+            if A is not None:
+                g = g + s * ((xf[t] @ A[e]) @ B[e])
+            gate, up = g[:I], g[I:]
+            h = np.array([gv / (1.0 + math.exp(-gv)) for gv in gate]) * up
+            out[t] += w[j] * (wdn @ h)
+    return out
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+def test_forward_equals_per_token_dense_loop(fmt):
+    E, H, I, k, T = 4, 64, 64, 2, 12
+    gu, dn = _tiny_layer(fmt, E, H, I)
+    x = synth.normal_bf16((T, H), 1.0, 0, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 0, "logits")
+    out, _ = moe.moe_forward(x, logits, k, fmt, E, H, I, gu[0], gu[1], dn[0], dn[1])
+    ref = _dense_loop(fmt, x, logits, k, E, H, I, gu, dn)
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
+
+
+def test_forward_with_one_expert_is_textbook_swiglu_ffn():
+    E, H, I, T = 1, 64, 128, 9
+    gu, dn = _tiny_layer("mxfp4", E, H, I, seed=3)
+    x = synth.normal_bf16((T, H), 1.0, 3, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 3, "logits")
+    out, _ = moe.moe_forward(x, logits, 1, "mxfp4", E, H, I, gu[0], gu[1], dn[0], dn[1])
+    X = bf16.bf16_bits_to_f64(x)
+    Wg = mxfp4.decode_mxfp4(gu[0], gu[1], 2 * I * H).reshape(2 * I, H)
+    Wd = mxfp4.decode_mxfp4(dn[0], dn[1], H * I).reshape(H, I)
+    gate, up = X @ Wg[:I].T, X @ Wg[I:].T
+    ffn = (gate * (1.0 / (1.0 + np.exp(-gate))) * up) @ Wd.T
+    assert np.allclose(out, ffn, rtol=1e-12, atol=1e-12 * np.abs(ffn).max())
+
+
+def test_forward_is_token_permutation_invariant():
+    E, H, I, k, T = 8, 64, 64, 3, 40
+    gu, dn = _tiny_layer("nf4", E, H, I, seed=7)
+    x = synth.normal_bf16((T, H), 1.0, 7, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 7, "logits")
+    out, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1])
+    p = np.random.default_rng(8).permutation(T)
+    outp, _ = moe.moe_forward(x[p], logits[p], k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1])
+    assert np.allclose(outp, out[p], rtol=1e-12, atol=1e-13 * np.abs(out).max())
+
+
+def test_forward_lora_zero_b_is_base_and_delta_matches_loop():
+    E, H, I, k, T, r = 4, 64, 64, 2, 10, 8
+    gu, dn = _tiny_layer("nf4", E, H, I, seed=9)
+    x = synth.normal_bf16((T, H), 1.0, 9, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 9, "logits")
+    A = synth.normal_bf16((E, H, r), 1.0 / r, 9, "A")
+    Bz = np.zeros((E, r, 2 * I), np.uint16)
+    base, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1])
+    zero, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1], A, Bz, 2.0)
+    assert np.array_equal(base, zero)
+    B = synth.normal_bf16((E, r, 2 * I), 0.01, 9, "B")
+    out, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1], A, B, 2.0)
+    ref = _dense_loop("nf4", x, logits, k, E, H, I, gu, dn,
+                      bf16.bf16_bits_to_f64(A).reshape(E, H, r), bf16.bf16_bits_to_f64(B).reshape(E, r, 2 * I), 2.0)
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
+    assert not np.allclose(out, base)
+
+
+def test_synth_is_deterministic_and_per_expert():
+    a = synth.stack_mxfp4(4, 32, 64, -6, 1, 0, "w")
+    b = synth.expert_mxfp4(2, 32, 64, -6, 1, 0, "w")
+    assert np.array_equal(a[0].reshape(4, -1)[2], b[0]) and np.array_equal(a[1].reshape(4, -1)[2], b[1])
+    sc = a[1]
+    assert sc.min() >= 127 - 6 and sc.max() <= 128
+    z = synth.zipf_logits_bf16(20000, 128, 1.1, 0, "z")
+    r = route.route(z[:4000], 4)
+    top = int(np.argmax(r["counts"]))
+    first = np.mean(r["ids"][:, 0] == top)     # first Gumbel-top-k draw follows p_e: ~0.226 for rank 1
+    assert 0.20 < first < 0.25
