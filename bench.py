@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Benchmark of the 4-bit routed-MoE layer forward on B200.
+
+One step is one forward of a Qwen3-30B-A3B-shaped NF4 MoE layer (E=128,
+H=2048, I=768, top-8) on a decode batch of T=64 tokens: routing, expert
+permute and gather, the grouped gate_up GEMM with in-kernel NF4 dequant and
+SwiGLU, the grouped down GEMM and the weighted combine.  Weights are seeded
+synthetic N(0, 0.02) values NF4-quantised on the device by the library's
+quantiser; activations and router logits are seeded N(0, 1) in bf16.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+the same workload instead (one token per step).  Under torchrun every rank
+runs an independent replica of the layer (the forward has no exchange step):
+``value`` is the whole-job token rate, timed on the device and taken as the
+max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "4-bit MoE layer tokens/s; decode weight GB/s vs HBM peak; prefill TFLOP/s"
+WORKLOAD = "qwen3_30b_a3b_nf4_decode"
+T_HEADLINE = 64
+L2_BYTES = 126 * 1000 * 1000
+KERNELS_PER_STEP = 6      # route_topk, route_rank, gather, gate_up GEMM, down GEMM, combine
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "bit_mixture_experts_top_b200", "csrc", "grouped_gemm.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_tag):
+    """DRAM bytes per launch of the kernel from the committed ncu summary, if it still matches the source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_tag)
+    if not e or e.get("source_digest") != source_digest():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler(threading.Thread):
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, gpu_index, period_s=0.002):
+        super().__init__(daemon=True)
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.stop_evt, self.err = period_s, threading.Event(), None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:          # no NVML: report the gap instead of guessing
+            self.nv, self.err = None, f"nvml unavailable: {e}"
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def run(self):
+        if self.nv is None:
+            return
+        while not self.stop_evt.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self._reasons()
+                for b, name in self.REASONS.items():
+                    if bits & b and b not in (0x1,):
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = str(e)
+            time.sleep(self.period)
+
+    def summary(self):
+        self.stop_evt.set()
+        self.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+                **({"note": self.err} if self.err else {})}
+
+
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def physical_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids) and ids[local].isdigit():
+            return int(ids[local])
+    return local
+
+
+def oracle_tokens_per_s(w, x, logits, rows, reps=1):
+    """Times the CPU oracle's forward on `rows` tokens (test infrastructure, baseline only)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import oracle_lora, oracle_stacks, touched_experts
+    from oracle import moe as omoe
+    experts = touched_experts(logits[rows], w.k)
+    stacks = oracle_stacks(w, experts)
+    A, B = oracle_lora(w)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        omoe.moe_forward(x[rows], logits[rows], w.k, w.fmt, w.E, w.H, w.I, *stacks, lora_A_bits=A, lora_B_bits=B,
+                         lora_scale=w.lora_scale)
+    dt = (time.perf_counter() - t0) / reps
+    return len(rows) / dt, dt, len(experts)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def bench_reference(args, world, rank):
+    """--impl reference: the oracle as it stands, one token of the workload per step, on host cores."""
+    if rank != 0:
+        return 0
+    from bit_mixture_experts_top_b200 import layer
+    from bit_mixture_experts_top_b200.workloads import WORKLOADS
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from helpers import oracle_stacks, touched_experts
+    from oracle import moe as omoe
+    w = WORKLOADS[WORKLOAD]
+    x, logits = layer.synthetic_tokens(w, T_HEADLINE)
+    steps, warmup = args.steps, args.warmup
+    rows = [i % T_HEADLINE for i in range(steps + warmup)]
+    stacks = oracle_stacks(w, touched_experts(logits[sorted(set(rows))], w.k))
+    for i in range(warmup):
+        omoe.moe_forward(x[rows[i]:rows[i] + 1], logits[rows[i]:rows[i] + 1], w.k, w.fmt, w.E, w.H, w.I, *stacks)
+    t0 = time.perf_counter()
+    for i in range(warmup, warmup + steps):
+        omoe.moe_forward(x[rows[i]:rows[i] + 1], logits[rows[i]:rows[i] + 1], w.k, w.fmt, w.E, w.H, w.I, *stacks)
+    dt = time.perf_counter() - t0
+    value = steps / dt
+    cores = blas_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": dt * 1e3 / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{WORKLOAD} T={T_HEADLINE} (one token per step)", "E": w.E, "H": w.H, "I": w.I,
+                   "k": w.k, "format": w.fmt, "global_batch": 1, "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "one token of the T=64 decode batch per step (8 routed experts decoded in fp64)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_e4b(args, world, rank, local):
+    import torch
+    from bit_mixture_experts_top_b200 import e4b, layer
+    from bit_mixture_experts_top_b200.workloads import WORKLOADS
+
+    dist = world > 1
+    if dist:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if dist else 0)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if dist:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v):
+        if not dist:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    w = WORKLOADS[WORKLOAD]
+    T = T_HEADLINE
+    lay = layer.synthetic_layer(w, dev)
+    x_np, lg_np = layer.synthetic_tokens(w, T)
+    x = layer.bits_tensor(x_np, dev)
+    lg = layer.bits_tensor(lg_np, dev)
+    out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+    ws = lay.workspace(T, dev)
+    args_fwd = (lay.desc, T, x, lg, lay.gate_up.codes, lay.gate_up.scales, lay.down.codes, lay.down.scales,
+                lay.lora_A, lay.lora_B, out, ws)
+
+    def step(ev_g0=None, ev_g1=None, ev_d1=None):
+        for st in (e4b.E4B_STAGE_ROUTE, e4b.E4B_STAGE_GATHER):
+            e4b.e4b_moe_forward_stage(st, *args_fwd)
+        if ev_g0 is not None:
+            ev_g0.record()
+        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_GATE_UP, *args_fwd)
+        if ev_g1 is not None:
+            ev_g1.record()
+        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_DOWN, *args_fwd)
+        if ev_d1 is not None:
+            ev_d1.record()
+        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_COMBINE, *args_fwd)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if e4b.e4b_device_status(ws) != e4b.E4B_OK:
+        raise RuntimeError("device status reported an error after warm-up")
+    offs = lay.region(T, e4b.E4B_WS_EXPERT_OFFSETS, torch.int32).cpu().numpy()
+    touched = int(np.count_nonzero(np.diff(offs)))
+    R = T * w.k
+    gu_bytes = touched * w.gate_up_bytes_per_expert() + R * w.H * 2 + R * w.I * 2
+    dn_bytes = touched * w.down_bytes_per_expert() + R * w.I * 2 + R * w.H * 4
+    layer_weight_bytes = touched * (w.gate_up_bytes_per_expert() + w.down_bytes_per_expert())
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(physical_gpu_index(local))
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start.record()
+    for i in range(K):
+        step(*evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.summary()
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    gu_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+    dn_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_per_step = max_over_ranks(total_ms / K)
+    gu_ms = max_over_ranks(gu_ms)
+    dn_ms = max_over_ranks(dn_ms)
+    if e4b.e4b_device_status(ws) != e4b.E4B_OK:
+        raise RuntimeError("device status reported an error in the timed region")
+
+    # end to end through the public call with host buffers: H2D inputs, forward, D2H output, every step
+    x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
+    lg_h = torch.from_numpy(lg_np.view(np.int16)).pin_memory()
+    out_h = torch.empty((T, w.H), dtype=torch.int16).pin_memory()
+    x_d = torch.empty((T, w.H), dtype=torch.int16, device=dev)
+    lg_d = torch.empty((T, w.E), dtype=torch.int16, device=dev)
+    out_d = torch.empty((T, w.H), dtype=torch.int16, device=dev)
+    e2e_steps = min(K, 200)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        lg_d.copy_(lg_h, non_blocking=True)
+        lay.forward(x_d, lg_d, out=out_d)
+        out_h.copy_(out_d, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    barrier()
+
+    peaks, peak_kind = load_peaks()
+    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    value = world * T / (ms_per_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD} T={T}", "E": w.E, "H": w.H, "I": w.I, "k": w.k, "format": w.fmt,
+                   "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {layer_weight_bytes / 1e6:.0f} MB of touched expert weights "
+                         f"per step vs {L2_BYTES / 1e6:.0f} MB L2, no flush"},
+        "roofline": {"bound": "hbm", "kernel": "grouped_gemm gate_up (NF4 dequant + SwiGLU)",
+                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_kind": peak_kind,
+                     "traffic": recorded_traffic("gate_up"),
+                     "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms},
+        "kernels": {"gate_up_ms": gu_ms, "down_ms": dn_ms,
+                    "down_gbs": dn_bytes / (dn_ms * 1e-3) / 1e9,
+                    "layer_weight_gbs": layer_weight_bytes / (ms_per_step * 1e-3) / 1e9,
+                    "touched_experts": touched},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_h.numel() * 2 + lg_h.numel() * 2),
+                "d2h_bytes_per_step": int(out_h.numel() * 2)},
+        "gpu_launches": K * KERNELS_PER_STEP,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, dt, ne = oracle_tokens_per_s(w, x_np, lg_np, np.arange(T), reps=2)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"the whole T={T} batch ({ne} experts decoded in fp64), "
+                                          f"timed twice, {dt:.1f} s per forward"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = init_dist()
+    if args.impl == "reference":
+        return bench_reference(args, world, rank)
+    return bench_e4b(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

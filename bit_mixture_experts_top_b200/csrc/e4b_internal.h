@@ -1,0 +1,87 @@
+// Host-side internals shared by the library's translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "e4b.h"
+
+namespace e4b {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxLoraRank = 16;
+constexpr int kRouteTokensPerBlock = 128;   // tokens per histogram block of the router
+constexpr int kStatusBytes = 256;           // status word + router done-counter at the start of a workspace
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded device waits: 2 s
+
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 16 fp32 NF4 levels and the 15 fp32 decision midpoints, built on the host from
+// the NormalFloat construction (own inverse-normal-CDF, see nf4_table.cpp).
+struct Nf4Table {
+  float level[16];
+  float mid[15];
+};
+const Nf4Table& nf4_table();
+
+// Router: status/done-counter layout inside the first kStatusBytes of a workspace.
+struct RouteBuffers {
+  int32_t* status;          // [2] device status word
+  uint32_t* done_counter;   // last-block detection of the histogram kernel
+  int32_t* topk_ids;        // [T*k]
+  float* topk_w;            // [T*k]
+  int32_t* expert_offsets;  // [E+1]
+  int32_t* chunk_off;       // [E+1] prefix of ceil(count_e / tokens_per_tile), or null
+  int32_t* block_counts;    // [nblk * E] per-block histograms, then per-block bases
+  int32_t* sorted_slot;     // [T*k]
+  int32_t* slot_pos;        // [T*k]
+};
+
+inline int route_blocks(int32_t T) { return (T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock; }
+
+cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t tokens_per_tile,
+                         const RouteBuffers& b, cudaStream_t s);
+
+cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n, uint16_t* out,
+                                 cudaStream_t s);
+
+cudaError_t launch_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, cudaStream_t s);
+
+// x_sorted[r] = x[sorted_slot[r] / k]; with LoRA also xa[r, j] = bf16(scale * x . A_e[:, j]) (j < r, zeros to 64).
+cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, const int32_t* sorted_slot,
+                          const int32_t* topk_ids, int32_t E, uint16_t* x_sorted, const uint16_t* lora_A,
+                          int32_t lora_rank, float lora_scale, uint16_t* xa, cudaStream_t s);
+
+// out[t] = sum_j w[t, j] * y[slot_pos[t*k + j]], j ascending, fp32 -> bf16.
+cudaError_t launch_combine(const float* y, const float* topk_w, const int32_t* slot_pos, int32_t T, int32_t k,
+                           int32_t H, uint16_t* out, cudaStream_t s);
+
+// Grouped 4-bit GEMMs on tcgen05.
+struct GroupedGemmLaunch {
+  int32_t mode;             // 0: gate_up + LoRA + SwiGLU -> bf16 h [R, I]; 1: down -> fp32 y [R, H]
+  int32_t fmt;              // E4B_NF4 / E4B_MXFP4
+  int32_t E, N, K, I;       // stack [E, N, K]; I = intermediate size (mode 0 pairing)
+  int32_t R;                // routed rows
+  int32_t tokens_per_tile;  // 32, 64, 128, 256
+  const uint8_t* codes;     // [E, N, K] packed
+  const void* scales;
+  const uint16_t* act;      // [R, K] bf16 (x_sorted or h)
+  const uint16_t* xa;       // [R, 64] bf16 LoRA left factor (mode 0) or null
+  const uint16_t* lora_B;   // [E, r, 2I] or null
+  int32_t lora_rank;
+  const int32_t* expert_offsets;
+  const int32_t* chunk_off;
+  void* out;                // mode 0: bf16 [R, I]; mode 1: fp32 [R, H]
+  int32_t* status;
+  uint64_t wait_limit_ns;
+};
+e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace e4b

@@ -1,0 +1,135 @@
+// Standalone format kernels: MXFP4 -> bf16 decode and the NF4 quantiser.
+//
+// Both are pure HBM streams.  Each warp owns a contiguous span of the flat
+// tensor, every lane moves 16 bytes per store (128-bit, fully coalesced), and
+// the grid is a multiple of the SM count with a grid-stride loop.
+//
+// MXFP4 decode ("How do I train and serve MoE models released in MXFP4 ...?",
+// "Why it happens" and "Two fidelity paths"): an E2M1 nibble
+// s.e1.e0.m is turned into an fp32 value exactly by placing its three
+// magnitude bits at fp32 bits 24..22 (which reads as e2m1 * 2^-126, subnormal
+// encoding included) and multiplying by 2^126; the E8M0 scale is the fp32
+// 2^(s-127) (s = 0 is the fp32 subnormal 2^-127, s = 255 NaN).  The product is
+// exact in fp32 and in bf16 unless it overflows, so one round-to-nearest
+// conversion reproduces the definition bit for bit.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+namespace {
+
+__device__ __forceinline__ float e2m1_to_f32(uint32_t nib) {
+  const uint32_t bits = ((nib & 8u) << 28) | ((nib & 7u) << 22);
+  return __uint_as_float(bits) * 0x1p126f;
+}
+
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  const uint32_t bits = (s == 0u) ? 0x00400000u : ((s == 255u) ? 0x7FC00000u : (s << 23));
+  return __uint_as_float(bits);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 8 elements = 4 code bytes -> 16 output bytes.  Unit u covers elements [8u, 8u+8).
+__global__ void __launch_bounds__(256) dequant_mxfp4_kernel(const uint32_t* __restrict__ codes,
+                                                              const uint8_t* __restrict__ scales, int64_t units,
+                                                              uint4* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units; u += stride) {
+    const uint32_t w = __ldcs(codes + u);
+    const uint32_t s = __ldg(scales + (u >> 2));
+    uint4 o;
+    if (s == 255u) {
+      o = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+    } else {
+      const float sc = e8m0_to_f32(s);
+      uint32_t r[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t byte = (w >> (8 * b)) & 0xFFu;
+        r[b] = pack_bf16x2(e2m1_to_f32(byte & 0xFu) * sc, e2m1_to_f32(byte >> 4) * sc);
+      }
+      o = make_uint4(r[0], r[1], r[2], r[3]);
+    }
+    __stcs(out + u, o);
+  }
+}
+
+struct Nf4Mids {
+  float m[15];
+};
+
+// One half-warp per 64-block: each lane loads 4 consecutive fp32 (16 bytes),
+// the half-warp reduces |x| to absmax, each lane emits 4 codes (2 bytes).
+__global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restrict__ x, int64_t quads,
+                                                             uint16_t* __restrict__ codes,
+                                                             float* __restrict__ absmax, Nf4Mids mids) {
+  __shared__ float s_mid[16];
+  if (threadIdx.x < 15) s_mid[threadIdx.x] = mids.m[threadIdx.x];
+  __syncthreads();
+  const float m7 = mids.m[7];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // quads is a multiple of 16, so every half-warp stays inside one block and
+  // the loop trip count is uniform across each half-warp.
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < quads; q += stride) {
+    const float4 v = __ldcs(x + q);
+    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16u);   // this half-warp only
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
+    uint32_t c[4];
+    const float xv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (a == 0.0f) {
+        c[i] = 7u;
+      } else {
+        const float y = __fdiv_rn(xv[i], a);
+        uint32_t k = (y > m7) ? 8u : 0u;        // count of midpoints below y, by bisection
+        k += (y > s_mid[k + 3]) ? 4u : 0u;
+        k += (y > s_mid[k + 1]) ? 2u : 0u;
+        k += (y > s_mid[k]) ? 1u : 0u;
+        c[i] = k;
+      }
+    }
+    const uint32_t b0 = (c[0] << 4) | c[1];
+    const uint32_t b1 = (c[2] << 4) | c[3];
+    codes[q] = static_cast<uint16_t>(b0 | (b1 << 8));
+    if ((threadIdx.x & 15) == 0) absmax[q >> 4] = a;
+  }
+}
+
+int grid_for(int64_t work_items, int threads, int per_sm) {
+  const int64_t need = (work_items + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * per_sm;
+  return static_cast<int>(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n, uint16_t* out,
+                                 cudaStream_t s) {
+  const int64_t units = n / 8;
+  if (units == 0) return cudaSuccess;
+  dequant_mxfp4_kernel<<<grid_for(units, 256, 8), 256, 0, s>>>(reinterpret_cast<const uint32_t*>(codes), scales,
+                                                              units, reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, cudaStream_t s) {
+  const int64_t quads = n / 4;
+  if (quads == 0) return cudaSuccess;
+  Nf4Mids m;
+  for (int i = 0; i < 15; ++i) m.m[i] = nf4_table().mid[i];
+  quantize_nf4_kernel<<<grid_for(quads, 256, 8), 256, 0, s>>>(reinterpret_cast<const float4*>(x), quads,
+                                                              reinterpret_cast<uint16_t*>(codes), absmax, m);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

@@ -1,0 +1,517 @@
+// Grouped 4-bit expert GEMMs on sm_100a tensor cores (tcgen05 / TMEM).
+//
+// What it computes (solutions index, grouped-nf4-gemm table: the routed MoE
+// expert GEMM straight on NF4 packed weights or on E2M1 blocks with E8M0
+// scales, one launch over all experts, fp32 accumulation, no bf16 expert
+// tensor; "experts4bit-qlora" limits list: the stock epilogue act(gate)*up;
+// experts4bit-qlora table of the index: ExpertsLoRA's per-expert low-rank
+// delta before the activation):
+//
+//   mode 0 (gate_up): G = X_e W_gu[e]^T (+ xa_e B_e), h = silu(G_gate) * G_up -> bf16 [R, I]
+//   mode 1 (down)   : Y = h_e W_dn[e]^T                                       -> fp32 [R, H]
+//
+// B200 design.  The weights are the UMMA M operand (128 rows per tile) and the
+// routed rows of one expert the N operand (tokens_per_tile = BN columns), so a
+// decode batch with a handful of rows per expert still issues full-height
+// MMAs, and one dequantised weight tile serves up to 256 rows in prefill.
+// One persistent CTA per SM walks a tile list (expert, weight block, row
+// chunk); consecutive tiles share a weight block so its bytes are read from
+// HBM once and from L2 after.  Warp roles:
+//   warp 0      TMA producer: packed codes (64-byte swizzled boxes) into a raw
+//               ring, activation tiles (128-byte swizzled) into the B ring;
+//   warp 1      TMEM owner and single-thread UMMA issuer (kind::f16, M=128,
+//               N=BN, K=16, fp32 accumulators in TMEM, two buffers);
+//   warps 2-9   dequant: 4-bit codes + per-block scale -> bf16 written in the
+//               128-byte-swizzled K-major layout the UMMA descriptor reads;
+//   warps 10-13 epilogue: tcgen05.ld, SwiGLU or fp32 store.
+// Every wait is bounded: on timeout the kernel records E4B_ERR_TIMEOUT, lets
+// copies and MMAs in flight land, frees its TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+namespace {
+
+constexpr int BM = 128;                      // weight rows per tile (UMMA M)
+constexpr int BK = 64;                       // K per MMA stage: one 128-byte swizzle row of bf16
+constexpr int RAW_K = 128;                   // K per packed-code stage
+constexpr int RAW_ROW_BYTES = RAW_K / 2;     // 64 bytes of codes per weight row
+constexpr int RAW_STAGE_BYTES = BM * RAW_ROW_BYTES;
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int NUM_DQ_WARPS = 8;
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int WARP_TMA = 0;
+constexpr int WARP_MMA = 1;
+constexpr int WARP_DQ0 = 2;
+constexpr int WARP_EPI0 = WARP_DQ0 + NUM_DQ_WARPS;
+constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
+
+template <int BN>
+struct Cfg {
+  static constexpr int B_STAGE_BYTES = BN * BK * 2;
+  static constexpr int STAGES = BN >= 256 ? 3 : (BN >= 128 ? 4 : 6);
+  static constexpr int RAW_STAGES = 6;
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_STAGE_BYTES;
+  static constexpr int OFF_RAW = OFF_B + STAGES * B_STAGE_BYTES;
+  static constexpr int OFF_BAR = OFF_RAW + RAW_STAGES * RAW_STAGE_BYTES;
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * RAW_STAGES + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_LUT = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_LUT + 64 + 1024;   // + slack to align the base to 1024
+  static_assert(B_STAGE_BYTES % 1024 == 0, "B stages must keep 1024-byte alignment");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+struct Params {
+  int32_t E, N, K, I;
+  int32_t n_blocks;       // weight blocks per expert (mode 0: I/64 gate+up pairs; mode 1: ceil(N/128))
+  int32_t ksteps;         // K / 64
+  int32_t lora_rank;      // 0 = none (mode 0 only)
+  const void* scales;
+  const uint16_t* lora_B; // [E, r, 2I]
+  const int32_t* expert_offsets;
+  const int32_t* chunk_off;
+  void* out;
+  int32_t* status;
+  uint64_t wait_limit_ns;
+  float lut[16];          // NF4 levels
+};
+
+struct Tile {
+  int e, nb, row0, rows;
+};
+
+template <int BN>
+__device__ __forceinline__ bool get_tile(const Params& p, int tile, int total, Tile& t) {
+  if (tile >= total) return false;
+  int lo = 0, hi = p.E;                 // last e with chunk_off[e] * n_blocks <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(p.chunk_off + mid) * p.n_blocks <= tile) lo = mid; else hi = mid;
+  }
+  const int c0 = __ldg(p.chunk_off + lo);
+  const int nch = __ldg(p.chunk_off + lo + 1) - c0;
+  const int local = tile - c0 * p.n_blocks;
+  t.e = lo;
+  t.nb = local / nch;
+  const int chunk = local - t.nb * nch;
+  const int off = __ldg(p.expert_offsets + lo);
+  t.row0 = off + chunk * BN;
+  t.rows = min(BN, __ldg(p.expert_offsets + lo + 1) - t.row0);
+  return true;
+}
+
+__device__ __forceinline__ float e2m1_to_f32(uint32_t nib) {
+  return __uint_as_float(((nib & 8u) << 28) | ((nib & 7u) << 22)) * 0x1p126f;
+}
+
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+  return __uint_as_float(s == 0u ? 0x00400000u : (s == 255u ? 0x7FC00000u : (s << 23)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 16 code bytes (32 elements, one scale) -> 4 x 16 bytes of bf16 in element order.
+template <int FMT>
+__device__ __forceinline__ void dequant32(const uint4 q, float sc, const float* lut, uint4 (&o)[4]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t r[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t byte = (w[i] >> (8 * b)) & 0xFFu;
+      float f0, f1;
+      if (FMT == E4B_NF4) {           // element 2j in the high nibble
+        f0 = lut[byte >> 4] * sc;
+        f1 = lut[byte & 0xFu] * sc;
+      } else {                        // MXFP4: element 2j in the low nibble
+        f0 = e2m1_to_f32(byte & 0xFu) * sc;
+        f1 = e2m1_to_f32(byte >> 4) * sc;
+      }
+      r[b] = pack_bf16x2(f0, f1);
+    }
+    o[i] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+template <int BN, int FMT, int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_act,
+                        const __grid_constant__ CUtensorMap tm_xa, const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sB = smem + C::OFF_B;
+  uint8_t* sRaw = smem + C::OFF_RAW;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* a_full = bars;
+  uint64_t* b_full = a_full + C::STAGES;
+  uint64_t* empty = b_full + C::STAGES;
+  uint64_t* raw_full = empty + C::STAGES;
+  uint64_t* raw_empty = raw_full + C::RAW_STAGES;
+  uint64_t* acc_full = raw_empty + C::RAW_STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int32_t* s_abort = reinterpret_cast<int32_t*>(smem + C::OFF_MISC + 8);
+  float* s_lut = reinterpret_cast<float*>(smem + C::OFF_LUT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&a_full[s], NUM_DQ_WARPS);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::RAW_STAGES; ++s) {
+      mbar_init(&raw_full[s], 1);
+      mbar_init(&raw_empty[s], NUM_DQ_WARPS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) s_lut[threadIdx.x] = p.lut[threadIdx.x];
+  if (warp == WARP_TMA && lane == 0) {
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_act);
+    if (MODE == 0 && p.lora_rank > 0) tma_prefetch_desc(&tm_xa);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(s_tmem, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *s_tmem;
+
+  const WaitCtx wctx{s_abort, p.status, p.wait_limit_ns};
+  const int total = __ldg(p.chunk_off + p.E) * p.n_blocks;
+  const bool lora = (MODE == 0) && p.lora_rank > 0;
+  const int nsteps = p.ksteps + (lora ? 1 : 0);
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0, rstage = 0;
+      uint32_t phase = 0, rphase = 0;
+      uint32_t armed_b = 0, armed_r = 0, par_b = 0, par_r = 0;   // per-stage "armed" bit and parity
+      bool ok = true;
+      Tile t;
+      for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x) {
+        for (int ks = 0; ks < nsteps; ++ks) {
+          if (ks < p.ksteps && (ks & 1) == 0) {
+            if (!mbar_wait(&raw_empty[rstage], rphase ^ 1u, wctx, 101)) { ok = false; break; }
+            mbar_arrive_expect_tx(&raw_full[rstage], RAW_STAGE_BYTES);
+            uint8_t* dst = sRaw + rstage * RAW_STAGE_BYTES;
+            const int x = ks * (BK / 2);
+            if (MODE == 0) {
+              tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + 64 * t.nb);
+              tma_load_2d(dst + 64 * RAW_ROW_BYTES, &tm_codes, &raw_full[rstage], x, t.e * p.N + p.I + 64 * t.nb);
+            } else {
+              tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + BM * t.nb);
+            }
+            armed_r |= 1u << rstage;
+            par_r = (par_r & ~(1u << rstage)) | (rphase << rstage);
+            if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
+          }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 102)) { ok = false; break; }
+          mbar_arrive_expect_tx(&b_full[stage], C::B_STAGE_BYTES);
+          if (ks < p.ksteps)
+            tma_load_2d(sB + stage * C::B_STAGE_BYTES, &tm_act, &b_full[stage], ks * BK, t.row0);
+          else
+            tma_load_2d(sB + stage * C::B_STAGE_BYTES, &tm_xa, &b_full[stage], 0, t.row0);
+          armed_b |= 1u << stage;
+          par_b = (par_b & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {   // let every issued copy land before the CTA's shared memory is released
+        for (int s = 0; s < C::RAW_STAGES; ++s)
+          if (armed_r & (1u << s)) mbar_drain(&raw_full[s], (par_r >> s) & 1u, kDrainNs);
+        for (int s = 0; s < C::STAGES; ++s)
+          if (armed_b & (1u << s)) mbar_drain(&b_full[s], (par_b >> s) & 1u, kDrainNs);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      uint64_t* last_bar = nullptr;
+      uint32_t last_par = 0;
+      Tile t;
+      for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t aphase = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[buf], aphase ^ 1u, wctx, 201)) { ok = false; break; }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+        for (int ks = 0; ks < nsteps; ++ks) {
+          if (!mbar_wait(&a_full[stage], phase, wctx, 202)) { ok = false; break; }
+          if (!mbar_wait(&b_full[stage], phase, wctx, 203)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_STAGE_BYTES);
+          const int nk = ks < p.ksteps ? BK / 16 : 1;       // the LoRA step is one K=16 MMA
+          for (int kk = 0; kk < nk; ++kk)
+            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+                         (ks > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          issued = true;
+          last_bar = &empty[stage];
+          last_par = phase;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+        last_bar = &acc_full[buf];
+        last_par = aphase;
+      }
+      if (!ok && issued) mbar_drain(last_bar, last_par, kDrainNs);   // MMAs in flight finish first
+    }
+  } else if (warp < WARP_EPI0) {
+    // ------------------------------------------------------------ dequant
+    const int dt = threadIdx.x - WARP_DQ0 * 32;   // 0..255
+    const int prow = dt & (BM - 1);               // A-tile row written by this thread
+    const int half = dt >> 7;                     // 32-element half of each 64-wide K stage
+    int stage = 0, rstage = 0;
+    uint32_t phase = 0, rphase = 0;
+    bool ok = true;
+    Tile t;
+    for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x) {
+      int raw_row, wrow;
+      if (MODE == 0) {                              // rows 32g..32g+15 gate, 32g+16..32g+31 up
+        const int g = prow >> 5, wi = prow & 31;
+        const int f = 64 * t.nb + 16 * g + (wi & 15);
+        raw_row = (wi < 16 ? 0 : 64) + 16 * g + (wi & 15);
+        wrow = (wi < 16) ? f : p.I + f;
+      } else {
+        raw_row = prow;
+        wrow = BM * t.nb + prow;
+      }
+      const int64_t grow = static_cast<int64_t>(t.e) * p.N + min(wrow, p.N - 1);
+      const float* sc_nf4 = reinterpret_cast<const float*>(p.scales) + grow * (p.K / 64);
+      const uint8_t* sc_mx = reinterpret_cast<const uint8_t*>(p.scales) + grow * (p.K / 32) + half;
+      auto load_scale = [&](int ks) -> float {
+        return FMT == E4B_NF4 ? __ldg(sc_nf4 + ks) : e8m0_to_f32(__ldg(sc_mx + 2 * ks));
+      };
+      float sc_next = load_scale(0);
+      for (int ks = 0; ks < p.ksteps; ++ks) {
+        const float sc = sc_next;
+        if (ks + 1 < p.ksteps) sc_next = load_scale(ks + 1);
+        if ((ks & 1) == 0 && !mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
+        if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
+        const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
+        const uint4 q = *reinterpret_cast<const uint4*>(
+            raw + swizzled_offset(raw_row, (ks & 1) * 2 + half, RAW_ROW_BYTES));
+        uint4 o[4];
+        dequant32<FMT>(q, sc, s_lut, o);
+        uint8_t* a = sA + stage * A_STAGE_BYTES;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        if ((ks & 1) == 1 || ks + 1 == p.ksteps) {
+          if (lane == 0) mbar_arrive(&raw_empty[rstage]);
+          if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
+        }
+      }
+      if (!ok) break;
+      if (lora) {                                   // A rows of the LoRA step: B_e[:, wrow]^T, rank padded to 16
+        if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 303)) { ok = false; break; }
+        if (half == 0) {
+          const uint16_t* bcol = p.lora_B + static_cast<int64_t>(t.e) * p.lora_rank * (2 * p.I) + wrow;
+          uint32_t v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t lo = (2 * j < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * j) * 2 * p.I) : 0u;
+            const uint32_t hi = (2 * j + 1 < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * j + 1) * 2 * p.I) : 0u;
+            v[j] = lo | (hi << 16);
+          }
+          uint8_t* a = sA + stage * A_STAGE_BYTES;
+          *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 0, 128)) = make_uint4(v[0], v[1], v[2], v[3]);
+          *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 1, 128)) = make_uint4(v[4], v[5], v[6], v[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[stage]);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                        // TMEM lanes 32q..32q+31
+    int it = 0;
+    Tile t;
+    for (int tile = blockIdx.x; get_tile<BN>(p, tile, total, t); tile += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t aphase = (it >> 1) & 1;
+      if (!mbar_wait(&acc_full[buf], aphase, wctx, 401)) break;
+      tc_fence_after_sync();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
+      for (int c0 = 0; c0 < BN && c0 < t.rows; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + c0, r);
+        tmem_ld_wait();
+        if (MODE == 0) {
+          const int f = 64 * t.nb + 16 * q + (lane & 15);
+          __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float v = __uint_as_float(r[j]);
+            const float u = __shfl_xor_sync(kFull, v, 16);
+            if (lane < 16 && c0 + j < t.rows) {
+              const float sg = __fdividef(v, 1.0f + __expf(-v));
+              h[static_cast<int64_t>(t.row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(sg * u);
+            }
+          }
+        } else {
+          const int n = BM * t.nb + 32 * q + lane;
+          float* y = reinterpret_cast<float*>(p.out);
+          if (n < p.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c0 + j < t.rows) y[static_cast<int64_t>(t.row0 + c0 + j) * p.N + n] = __uint_as_float(r[j]);
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int FMT, int MODE>
+e4b_status launch_typed(const GroupedGemmLaunch& g, const CUtensorMap& tc, const CUtensorMap& ta,
+                        const CUtensorMap& tx, const Params& prm, cudaStream_t s) {
+  using C = Cfg<BN>;
+  auto kern = grouped_gemm_kernel<BN, FMT, MODE>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return E4B_ERR_CUDA;
+  const int64_t active = g.R < g.E ? g.R : g.E;
+  const int64_t max_tiles = (active + (g.R + BN - 1) / BN) * prm.n_blocks;
+  const int64_t sms = device_sm_count();
+  const int grid = static_cast<int>(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
+  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, s>>>(tc, ta, tx, prm);
+  return cudaGetLastError() == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+}
+
+template <int BN>
+e4b_status dispatch_fmt_mode(const GroupedGemmLaunch& g, const CUtensorMap& tc, const CUtensorMap& ta,
+                             const CUtensorMap& tx, const Params& prm, cudaStream_t s) {
+  if (g.fmt == E4B_NF4)
+    return g.mode == 0 ? launch_typed<BN, E4B_NF4, 0>(g, tc, ta, tx, prm, s)
+                       : launch_typed<BN, E4B_NF4, 1>(g, tc, ta, tx, prm, s);
+  return g.mode == 0 ? launch_typed<BN, E4B_MXFP4, 0>(g, tc, ta, tx, prm, s)
+                     : launch_typed<BN, E4B_MXFP4, 1>(g, tc, ta, tx, prm, s);
+}
+
+}  // namespace
+
+e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
+  if (g.R == 0) return E4B_OK;
+  const int BN = g.tokens_per_tile;
+  CUtensorMap tc, ta, tx;
+  const uint64_t code_rows = static_cast<uint64_t>(g.E) * g.N;
+  if (!encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, RAW_ROW_BYTES,
+                 g.mode == 0 ? 64 : BM, CU_TENSOR_MAP_SWIZZLE_64B))
+    return E4B_ERR_CUDA;
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, BK, BN,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return E4B_ERR_CUDA;
+  const bool lora = g.mode == 0 && g.lora_rank > 0;
+  if (lora) {
+    if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.xa, 64, g.R, 128, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+      return E4B_ERR_CUDA;
+  } else {
+    tx = ta;
+  }
+  Params prm;
+  prm.E = g.E;
+  prm.N = g.N;
+  prm.K = g.K;
+  prm.I = g.I;
+  prm.n_blocks = g.mode == 0 ? g.I / 64 : (g.N + BM - 1) / BM;
+  prm.ksteps = g.K / BK;
+  prm.lora_rank = lora ? g.lora_rank : 0;
+  prm.scales = g.scales;
+  prm.lora_B = g.lora_B;
+  prm.expert_offsets = g.expert_offsets;
+  prm.chunk_off = g.chunk_off;
+  prm.out = g.out;
+  prm.status = g.status;
+  prm.wait_limit_ns = g.wait_limit_ns;
+  for (int i = 0; i < 16; ++i) prm.lut[i] = nf4_table().level[i];
+  switch (BN) {
+    case 32: return dispatch_fmt_mode<32>(g, tc, ta, tx, prm, s);
+    case 64: return dispatch_fmt_mode<64>(g, tc, ta, tx, prm, s);
+    case 128: return dispatch_fmt_mode<128>(g, tc, ta, tx, prm, s);
+    case 256: return dispatch_fmt_mode<256>(g, tc, ta, tx, prm, s);
+    default: return E4B_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace e4b

@@ -1,0 +1,293 @@
+// Top-k routing, expert histogram, stable expert permute, row gather (with the
+// LoRA left factor) and the weighted combine.
+//
+// Routing (solutions index, grouped-nf4-gemm table: the routed expert GEMM runs
+// over all experts in one launch, so routed rows are grouped by expert first;
+// "experts4bit-qlora", "Current measured position": routing is decided on the
+// router logits):
+//   * one warp per token; lane l holds the logits of experts l, l+32, ...
+//     packed into 32-bit keys (order-preserving bf16 bits << 16 | 0xFFFF - id),
+//     so one unsigned max picks the largest logit and, on ties, the lowest id;
+//     k rounds of __reduce_max_sync select the k experts;
+//   * gate weights are the fp32 softmax of the k selected logits;
+//   * the block histogram feeds per-block counts; the last block to finish
+//     turns them into expert offsets, per-block bases and tile-chunk offsets;
+//   * the rank kernel orders each block's slots by (expert, slot) with
+//     warp-level __match_any_sync ranks, which makes the permute stable and
+//     deterministic.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "e4b_device.cuh"
+#include "e4b_internal.h"
+
+namespace e4b {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+__device__ __forceinline__ uint32_t route_key(uint16_t bits, int e) {
+  if (bits == 0x8000u) bits = 0;                                    // -0 == +0
+  const uint32_t ord = (bits & 0x8000u) ? (~bits & 0xFFFFu) : (bits | 0x8000u);
+  return (ord << 16) | (0xFFFFu - static_cast<uint32_t>(e));
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+__global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E, int k,
+                                                              int tokens_per_tile, int nblk,
+                                                              int32_t* __restrict__ topk_ids,
+                                                              float* __restrict__ topk_w, int32_t* block_counts,
+                                                              uint32_t* done_counter, int32_t* expert_offsets,
+                                                              int32_t* chunk_off) {
+  __shared__ int32_t s_cnt[kMaxExperts];
+  __shared__ int32_t s_tot[kMaxExperts + 1];
+  __shared__ bool s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += kThreads) s_cnt[e] = 0;
+  __syncthreads();
+
+  const int t_begin = blockIdx.x * kRouteTokensPerBlock;
+  const int per_lane = (E + 31) >> 5;      // <= 8
+  for (int tt = warp; tt < kRouteTokensPerBlock; tt += kWarps) {
+    const int t = t_begin + tt;
+    if (t >= T) break;
+    const uint16_t* row = logits + static_cast<int64_t>(t) * E;
+    uint32_t key[kMaxExperts / 32];
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane + 32 * j;
+      key[j] = (j < per_lane && e < E) ? route_key(row[e], e) : 0u;   // real keys are never 0
+    }
+    uint32_t mine = 0;                     // lane j keeps the j-th pick
+    for (int r = 0; r < k; ++r) {
+      uint32_t best = 0;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[j]);
+      best = __reduce_max_sync(kFull, best);
+      const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j)
+        if (lane + 32 * j == e) key[j] = 0u;
+      if (lane == r) mine = best;
+    }
+    int id = 0;
+    float v = 0.0f;
+    if (lane < k) {
+      id = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
+      v = bf16_bits_to_f32(row[id]);
+    }
+    const float m = __shfl_sync(kFull, v, 0);          // the first pick holds the maximum
+    float ex = (lane < k) ? expf(v - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    if (lane < k) {
+      topk_ids[static_cast<int64_t>(t) * k + lane] = id;
+      topk_w[static_cast<int64_t>(t) * k + lane] = ex / sum;
+      atomicAdd(&s_cnt[id], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kThreads) block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = s_cnt[e];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(done_counter, 1u) == static_cast<uint32_t>(nblk - 1));
+  __syncthreads();
+  if (!s_last) return;
+
+  // Last block: totals, exclusive offsets, per-block bases, tile-chunk offsets.
+  __threadfence();
+  for (int e = tid; e < E; e += kThreads) {
+    int32_t tot = 0;
+    for (int b = 0; b < nblk; ++b) tot += __ldcg(block_counts + static_cast<int64_t>(b) * E + e);
+    s_tot[e] = tot;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0, crun = 0;
+    for (int e = 0; e < E; ++e) {
+      const int32_t c = s_tot[e];
+      expert_offsets[e] = run;
+      if (chunk_off) chunk_off[e] = crun;
+      s_tot[e] = run;
+      run += c;
+      if (tokens_per_tile > 0) crun += (c + tokens_per_tile - 1) / tokens_per_tile;
+    }
+    expert_offsets[E] = run;
+    if (chunk_off) chunk_off[E] = crun;
+    *done_counter = 0u;                               // ready for the next call
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kThreads) {
+    int32_t run = s_tot[e];
+    for (int b = 0; b < nblk; ++b) {
+      int32_t* p = block_counts + static_cast<int64_t>(b) * E + e;
+      const int32_t c = __ldcg(p);
+      *p = run;                                       // becomes block b's base for expert e
+      run += c;
+    }
+  }
+}
+
+// Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
+// slots of the block with the same expert).  Each warp owns a contiguous
+// segment; per-warp histograms are scanned across warps first.
+__global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __restrict__ topk_ids, int T, int E,
+                                                              int k, const int32_t* __restrict__ block_base,
+                                                              int32_t* __restrict__ sorted_slot,
+                                                              int32_t* __restrict__ slot_pos) {
+  __shared__ int32_t s_wc[kWarps][kMaxExperts];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock * k;
+  const int64_t s1 = min(static_cast<int64_t>(T), static_cast<int64_t>(blockIdx.x + 1) * kRouteTokensPerBlock) * k;
+  const int64_t n = s1 - s0;
+  const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t w0 = s0 + warp * seg, w1 = min(s1, w0 + seg);
+  for (int i = tid; i < kWarps * kMaxExperts; i += kThreads) (&s_wc[0][0])[i] = 0;
+  __syncthreads();
+  for (int64_t s = w0 + lane; s < w1; s += 32) atomicAdd(&s_wc[warp][topk_ids[s]], 1);
+  __syncthreads();
+  for (int e = tid; e < E; e += kThreads) {
+    int32_t run = block_base[static_cast<int64_t>(blockIdx.x) * E + e];
+    for (int w = 0; w < kWarps; ++w) {
+      const int32_t c = s_wc[w][e];
+      s_wc[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t c0 = w0; c0 < w1; c0 += 32) {
+    const int64_t s = c0 + lane;
+    const bool valid = s < w1;
+    const int id = valid ? topk_ids[s] : (kMaxExperts + lane);   // invalid lanes never match
+    const uint32_t peers = __match_any_sync(kFull, id);
+    const int rank = __popc(peers & lt);
+    int32_t pos = 0;
+    if (valid) pos = s_wc[warp][id] + rank;
+    __syncwarp();
+    if (valid && rank == __popc(peers) - 1) s_wc[warp][id] += __popc(peers);
+    __syncwarp();
+    if (valid) {
+      sorted_slot[pos] = static_cast<int32_t>(s);
+      slot_pos[s] = pos;
+    }
+  }
+}
+
+// One warp per routed row: copy the token's activations into expert order and,
+// with LoRA, form xa = scale * x . A_e (bf16, rank padded with zeros to 64).
+__global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __restrict__ x, int H, int k, int R,
+                                                          const int32_t* __restrict__ sorted_slot,
+                                                          const int32_t* __restrict__ topk_ids,
+                                                          uint16_t* __restrict__ x_sorted,
+                                                          const uint16_t* __restrict__ lora_A, int rank,
+                                                          float scale, uint16_t* __restrict__ xa) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  if (r >= R) return;
+  const int32_t slot = sorted_slot[r];
+  const int64_t t = slot / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+  uint4* dst = reinterpret_cast<uint4*>(x_sorted + r * H);
+  const int nvec = H / 8;
+  float acc[kMaxLoraRank];
+#pragma unroll
+  for (int j = 0; j < kMaxLoraRank; ++j) acc[j] = 0.0f;
+  const uint16_t* Ae = lora_A ? lora_A + static_cast<int64_t>(topk_ids[slot]) * H * rank : nullptr;
+  for (int v = lane; v < nvec; v += 32) {
+    const uint4 q = __ldg(src + v);
+    dst[v] = q;
+    if (Ae) {
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float xv = bf16_bits_to_f32(static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1))));
+        const uint16_t* arow = Ae + static_cast<int64_t>(v * 8 + i) * rank;
+#pragma unroll
+        for (int j = 0; j < kMaxLoraRank; ++j)
+          if (j < rank) acc[j] = fmaf(xv, bf16_bits_to_f32(__ldg(arow + j)), acc[j]);
+      }
+    }
+  }
+  if (!Ae) return;
+#pragma unroll
+  for (int j = 0; j < kMaxLoraRank; ++j) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(kFull, acc[j], off);
+  }
+  // lane l writes columns 2l, 2l+1 of the 64-wide row
+  float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+  for (int j = 0; j < kMaxLoraRank; ++j) {
+    if (j < rank && j == 2 * lane) lo = acc[j] * scale;
+    if (j < rank && j == 2 * lane + 1) hi = acc[j] * scale;
+  }
+  __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
+  reinterpret_cast<uint32_t*>(xa + r * 64)[lane] = *reinterpret_cast<uint32_t*>(&pr);
+}
+
+// One block per token: out[t] = sum_j w[t, j] * y[slot_pos[t*k + j]], j ascending.
+__global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ y,
+                                                           const float* __restrict__ topk_w,
+                                                           const int32_t* __restrict__ slot_pos, int k, int H,
+                                                           uint16_t* __restrict__ out) {
+  const int64_t t = blockIdx.x;
+  const int nq = H / 4;
+  for (int c = threadIdx.x; c < nq; c += kThreads) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float w = __ldg(topk_w + t * k + j);
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(y + static_cast<int64_t>(__ldg(slot_pos + t * k + j)) * H) + c);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 o = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+    reinterpret_cast<uint2*>(out + t * H)[c] = o;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t tokens_per_tile,
+                         const RouteBuffers& b, cudaStream_t s) {
+  if (T == 0) {
+    cudaError_t err = cudaMemsetAsync(b.expert_offsets, 0, sizeof(int32_t) * (E + 1), s);
+    if (err == cudaSuccess && b.chunk_off) err = cudaMemsetAsync(b.chunk_off, 0, sizeof(int32_t) * (E + 1), s);
+    return err;
+  }
+  const int nblk = route_blocks(T);
+  route_topk_kernel<<<nblk, kThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
+                                               b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  route_rank_kernel<<<nblk, kThreads, 0, s>>>(b.topk_ids, T, E, k, b.block_counts, b.sorted_slot, b.slot_pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, const int32_t* sorted_slot,
+                          const int32_t* topk_ids, int32_t E, uint16_t* x_sorted, const uint16_t* lora_A,
+                          int32_t lora_rank, float lora_scale, uint16_t* xa, cudaStream_t s) {
+  (void)E;
+  if (R == 0) return cudaSuccess;
+  const int grid = (R + kWarps - 1) / kWarps;
+  gather_kernel<<<grid, kThreads, 0, s>>>(x, H, k, R, sorted_slot, topk_ids, x_sorted, lora_A, lora_rank,
+                                          lora_scale, xa);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* y, const float* topk_w, const int32_t* slot_pos, int32_t T, int32_t k,
+                           int32_t H, uint16_t* out, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  combine_kernel<<<T, kThreads, 0, s>>>(y, topk_w, slot_pos, k, H, out);
+  return cudaGetLastError();
+}
+
+}  // namespace e4b

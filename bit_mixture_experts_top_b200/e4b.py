@@ -1,0 +1,180 @@
+"""Python binding of the C ABI in ``include/e4b.h`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does
+nothing but pass device pointers, sizes and the current CUDA stream; all
+arithmetic runs in the library's kernels.  Tensors must already live on the
+GPU.  If ``libe4b.so`` is missing or cannot be loaded, :func:`lib` raises --
+there is no fallback path.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libe4b.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "e4b.h")
+
+E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_UNSUPPORTED, E4B_ERR_CUDA, E4B_ERR_TIMEOUT = range(5)
+E4B_NF4, E4B_MXFP4 = 0, 1
+E4B_ACT_SWIGLU = 0
+E4B_STAGE_ROUTE, E4B_STAGE_GATHER, E4B_STAGE_GATE_UP, E4B_STAGE_DOWN, E4B_STAGE_COMBINE = range(5)
+(E4B_WS_TOPK_IDS, E4B_WS_TOPK_W, E4B_WS_EXPERT_OFFSETS, E4B_WS_SORTED_SLOT, E4B_WS_X_SORTED, E4B_WS_H,
+ E4B_WS_Y) = range(7)
+FORMATS = {"nf4": E4B_NF4, "mxfp4": E4B_MXFP4}
+
+
+class E4BError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {lib().e4b_status_string(status).decode()}")
+
+
+class MoeDesc(ctypes.Structure):
+    _fields_ = [
+        ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("k", ctypes.c_int32),
+        ("format", ctypes.c_int32), ("lora_rank", ctypes.c_int32), ("lora_scale", ctypes.c_float),
+        ("act", ctypes.c_int32), ("tokens_per_tile", ctypes.c_int32),
+    ]
+
+
+def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0):
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_SWIGLU, tokens_per_tile)
+
+
+_LIB = None
+_vp, _sz, _i32, _i64, _u32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
+_SIGS = {
+    "e4b_abi_version": ([], _i32),
+    "e4b_status_string": ([_i32], ctypes.c_char_p),
+    "e4b_nf4_codebook": ([_vp], None),
+    "e4b_dequant_mxfp4": ([_vp, _vp, _i64, _vp, _vp], _i32),
+    "e4b_quantize_nf4": ([_vp, _i64, _vp, _vp, _vp], _i32),
+    "e4b_route_workspace_bytes": ([_i32, _i32, _i32], _sz),
+    "e4b_route": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_moe_workspace_bytes": ([ctypes.POINTER(MoeDesc), _i32], _sz),
+    "e4b_moe_workspace_region": ([ctypes.POINTER(MoeDesc), _i32, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz)], _i32),
+    "e4b_moe_forward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_moe_forward_stage": ([_i32, ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _sz, _vp], _i32),
+    "e4b_device_status": ([_vp, _vp], _i32),
+    "e4b_debug_wait_timeout": ([_u32, _vp, _sz, _vp], _i32),
+}
+
+
+def lib():
+    """The loaded library; raises if it was not built or cannot be loaded."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m bit_mixture_experts_top_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def header_functions():
+    """Names of the functions include/e4b.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(e4b_[a-z0-9_]+)\s*\(", text)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status, where):
+    if status != E4B_OK:
+        raise E4BError(status, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("e4b: tensors must be CUDA tensors")
+
+
+# ---------------------------------------------------------------------------- entry points
+
+def e4b_abi_version():
+    return lib().e4b_abi_version()
+
+
+def e4b_nf4_codebook():
+    import numpy as np
+    out = (ctypes.c_float * 16)()
+    lib().e4b_nf4_codebook(out)
+    return np.frombuffer(out, dtype=np.float32).copy()
+
+
+def e4b_dequant_mxfp4(codes, scales, n, out, stream=None):
+    _need_cuda(codes, scales, out)
+    _check(lib().e4b_dequant_mxfp4(_ptr(codes), _ptr(scales), n, _ptr(out), _stream(stream)), "e4b_dequant_mxfp4")
+    return out
+
+
+def e4b_quantize_nf4(x, n, codes, absmax, stream=None):
+    _need_cuda(x, codes, absmax)
+    _check(lib().e4b_quantize_nf4(_ptr(x), n, _ptr(codes), _ptr(absmax), _stream(stream)), "e4b_quantize_nf4")
+    return codes, absmax
+
+
+def e4b_route_workspace_bytes(T, E, k):
+    return lib().e4b_route_workspace_bytes(T, E, k)
+
+
+def e4b_route(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_slot, ws, stream=None):
+    _need_cuda(logits, topk_ids, topk_w, expert_offsets, sorted_slot, ws)
+    _check(lib().e4b_route(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
+                           _ptr(sorted_slot), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "e4b_route")
+
+
+def e4b_moe_workspace_bytes(desc, T):
+    return lib().e4b_moe_workspace_bytes(ctypes.byref(desc), T)
+
+
+def e4b_moe_workspace_region(desc, T, region):
+    off, nbytes = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().e4b_moe_workspace_region(ctypes.byref(desc), T, region, ctypes.byref(off), ctypes.byref(nbytes)),
+           "e4b_moe_workspace_region")
+    return off.value, nbytes.value
+
+
+def e4b_moe_forward(desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, out, ws,
+                    stream=None):
+    _need_cuda(x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, out, ws)
+    _check(lib().e4b_moe_forward(ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(gu_codes), _ptr(gu_scales),
+                                 _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B), _ptr(out), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "e4b_moe_forward")
+    return out
+
+
+def e4b_moe_forward_stage(stage, desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B,
+                          out, ws, stream=None):
+    _check(lib().e4b_moe_forward_stage(stage, ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(gu_codes),
+                                       _ptr(gu_scales), _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B),
+                                       _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "e4b_moe_forward_stage")
+    return out
+
+
+def e4b_device_status(ws, stream=None):
+    """Synchronises the stream and returns (and clears) the workspace's device status code."""
+    return lib().e4b_device_status(_ptr(ws), _stream(stream))
+
+
+def e4b_debug_wait_timeout(limit_ns, ws, stream=None):
+    _check(lib().e4b_debug_wait_timeout(limit_ns, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "e4b_debug_wait_timeout")

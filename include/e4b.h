@@ -1,0 +1,234 @@
+/*
+ * e4b.h -- C ABI of the 4-bit routed-MoE layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The library computes the forward of one routed Mixture-of-Experts layer
+ * whose fused expert stacks [E, ...] stay packed in 4-bit, as NF4 or MXFP4,
+ * plus the two standalone format kernels (MXFP4 -> bf16 decode and the NF4
+ * quantiser).  Sources for what each call computes, by page and section:
+ *
+ *   [MX]  "How do I train and serve MoE models released in MXFP4 (gpt-oss,
+ *         DeepSeek-V4)?" -- "Why it happens" (MXFP4: two E2M1 nibbles per
+ *         byte, 32-value blocks sharing one E8M0 power-of-two scale) and
+ *         "Two fidelity paths" (bit-exact MXFP4 decode; Experts4bit.from_float
+ *         quantises a float stack to NF4).
+ *   [IX]  "MoE Training & Inference Guides" (solutions index) --
+ *         grouped-nf4-gemm table: the routed MoE expert GEMM on NF4 packed
+ *         weights (gemm_4bit_grouped) and on E2M1/E8M0 bytes
+ *         (gemm_mxfp4_grouped), one launch over all experts, fp32
+ *         accumulation, no bf16 expert tensor; experts4bit-qlora table:
+ *         ExpertsLoRA, a per-expert low-rank delta before each routed
+ *         expert's activation.
+ *   [PKG] "experts4bit-qlora" package page -- limits list: one fp32 absmax
+ *         per 64 NF4 weights; the stock expert epilogue act(gate)*up with no
+ *         biases or clamps; "Current measured position": routing is decided
+ *         on the router logits.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are plain CUDA device addresses; the caller owns every
+ *     buffer.  The library never allocates memory; scratch lives in a
+ *     caller-provided workspace whose size the *_workspace_bytes queries give.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Calls return before the GPU finishes.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return E4B_ERR_INVALID_ARG or E4B_ERR_UNSUPPORTED; nothing is
+ *     enqueued then.  A failed launch returns E4B_ERR_CUDA.  Kernels never
+ *     trap: a bounded wait that runs out records E4B_ERR_TIMEOUT in the
+ *     workspace status word, which e4b_device_status() reports.
+ *   - There is no fallback path: a call either runs these kernels or fails.
+ *
+ * Storage layouts (readings of the pages where they are silent):
+ *   - Expert stacks are stored K-contiguous: gate_up as [E, 2I, H] (logical
+ *     [E, H, 2I] transposed), down as [E, H, I]; the fused 2I rows are
+ *     [gate rows 0..I-1 | up rows I..2I-1].  Quantisation blocks are runs of
+ *     the flat stored stack, hence along K.
+ *   - MXFP4: element 2j is the LOW nibble of byte j; scale byte b covers
+ *     elements [32b, 32b+32); value = e2m1(code) * 2^(scale - 127), 0xFF = NaN.
+ *   - NF4: element 2j is the HIGH nibble of byte j; absmax[b] (fp32) covers
+ *     elements [64b, 64b+64); value = level[code] * absmax.
+ */
+#ifndef E4B_H
+#define E4B_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define E4B_ABI_VERSION 1
+
+typedef enum {
+  E4B_OK = 0,
+  E4B_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, workspace too small */
+  E4B_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement */
+  E4B_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  E4B_ERR_TIMEOUT = 4        /* a bounded device-side wait ran out (reported by e4b_device_status) */
+} e4b_status;
+
+enum { E4B_NF4 = 0, E4B_MXFP4 = 1 };   /* e4b_moe_desc.format */
+enum { E4B_ACT_SWIGLU = 0 };           /* e4b_moe_desc.act: h = silu(gate) * up */
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* e4b_stream;
+
+/* One MoE layer.  [IX] (grouped GEMMs, ExpertsLoRA), [PKG] (stock epilogue). */
+typedef struct {
+  int32_t E;               /* experts, 1..256 */
+  int32_t H;               /* hidden size, multiple of 64 */
+  int32_t I;               /* expert intermediate size, multiple of 64 */
+  int32_t k;               /* experts per token, 1..min(E, 32) */
+  int32_t format;          /* E4B_NF4 or E4B_MXFP4 */
+  int32_t lora_rank;       /* 0 = no LoRA; else 1..16 */
+  float lora_scale;        /* alpha / r, multiplies the LoRA delta */
+  int32_t act;             /* E4B_ACT_SWIGLU */
+  int32_t tokens_per_tile; /* 0 = chosen by the library; else 32, 64, 128 or 256 */
+} e4b_moe_desc;
+
+/* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */
+int32_t e4b_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char* e4b_status_string(int32_t status);
+
+/* The library's 16 NF4 levels (ascending, fp32), as its kernels use them.
+ * Host-only; out must hold 16 floats.  [PKG]/[IX]: NormalFloat levels. */
+void e4b_nf4_codebook(float* out);
+
+/*
+ * Standalone MXFP4 -> bf16 decode.  [MX] "Two fidelity paths": exact decode
+ * of the released blocks and scales.
+ *   codes  : n/2 bytes, 16-byte aligned       (device, read)
+ *   scales : n/32 E8M0 bytes                  (device, read)
+ *   n      : element count, multiple of 32, >= 0
+ *   out    : n bf16 values, 16-byte aligned   (device, written)
+ * Bit-exact: out[i] = bf16(e2m1(code_i) * 2^(scales[i/32] - 127)); the
+ * product is exact unless it overflows (+-inf); scale 0xFF gives NaN.
+ */
+e4b_status e4b_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n,
+                             uint16_t* out, e4b_stream stream);
+
+/*
+ * Standalone NF4 quantiser (Experts4bit.from_float).  [MX] "Two fidelity
+ * paths"; [PKG] one fp32 absmax per 64 weights.
+ *   x      : n fp32 values, 16-byte aligned   (device, read)
+ *   n      : multiple of 64, >= 0
+ *   codes  : n/2 bytes, packed high nibble first (device, written)
+ *   absmax : n/64 fp32                        (device, written)
+ * Per 64-block: a = max|x| (exact); a == 0 gives code 7 everywhere; else
+ * y = x / a (IEEE fp32 division) and code = #{i : y > m_i} with the fp32
+ * midpoints m_i = fl32((level_i + level_{i+1}) / 2).  NaN/Inf input is
+ * outside the contract.
+ */
+e4b_status e4b_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax,
+                            e4b_stream stream);
+
+/* Workspace bytes e4b_route needs for T tokens, E experts, k choices. */
+size_t e4b_route_workspace_bytes(int32_t T, int32_t E, int32_t k);
+
+/*
+ * Top-k routing and expert permute.  [IX] (routed expert GEMM over all
+ * experts in one launch), [PKG] "Current measured position" (routing is
+ * defined on given logits).
+ *   logits         : [T, E] bf16, row-major       (device, read)
+ *   topk_ids       : [T, k] int32                 (device, written) ids by
+ *                    (logit desc, id asc); -0 == +0
+ *   topk_w         : [T, k] fp32                  (device, written) softmax of
+ *                    the k selected logits
+ *   expert_offsets : [E+1] int32                  (device, written) exclusive
+ *                    prefix sum of per-expert slot counts
+ *   sorted_slot    : [T*k] int32                  (device, written) slots
+ *                    s = t*k + j grouped by expert, ascending s in each group
+ *   ws, ws_bytes   : workspace, 256-byte aligned, >= e4b_route_workspace_bytes
+ * Integer outputs are deterministic and bit-exact.  T == 0 is a no-op that
+ * still writes expert_offsets (all zero).
+ */
+e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
+                     int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                     int32_t* sorted_slot, void* ws, size_t ws_bytes, e4b_stream stream);
+
+/* Workspace bytes e4b_moe_forward needs for this layer at T tokens (0 on a bad desc). */
+size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
+
+/*
+ * Layer forward.  [IX] grouped gate_up GEMM with in-kernel dequant, optional
+ * per-expert LoRA delta before the activation, [PKG] SwiGLU epilogue
+ * act(gate)*up, grouped down GEMM, then the weighted combine
+ * out[t] = sum_j w[t,j] * y[t,j] in fp32, j ascending, rounded to bf16.
+ *   x         : [T, H] bf16                            (device, read)
+ *   logits    : [T, E] bf16                            (device, read)
+ *   gu_codes  : [E, 2I, H] packed 4-bit (E*2I*H/2 bytes, 16-byte aligned)
+ *   gu_scales : NF4 fp32 absmax [E*2I*H/64] or MXFP4 E8M0 bytes [E*2I*H/32]
+ *   dn_codes  : [E, H, I] packed 4-bit;  dn_scales as gu_scales for [E, H, I]
+ *   lora_A    : [E, H, r] bf16 or NULL;  lora_B : [E, r, 2I] bf16 or NULL
+ *               (both or neither, and r == d->lora_rank)
+ *   out       : [T, H] bf16                            (device, written)
+ *   ws        : workspace, 256-byte aligned, >= e4b_moe_workspace_bytes(d, T);
+ *               its first 256 bytes hold the device status word
+ * bf16 outputs match the fp64 definition within relative Frobenius error
+ * 5e-3 and max-abs error 3e-2 * max|ref|; routing is bit-exact.
+ */
+e4b_status e4b_moe_forward(const e4b_moe_desc* d, int32_t T, const uint16_t* x,
+                           const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
+                           const uint8_t* dn_codes, const void* dn_scales,
+                           const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* out,
+                           void* ws, size_t ws_bytes, e4b_stream stream);
+
+/* Stages of e4b_moe_forward, in order. */
+enum {
+  E4B_STAGE_ROUTE = 0,     /* clears the status word; top-k, histogram, stable permute */
+  E4B_STAGE_GATHER = 1,    /* routed rows in expert order (+ LoRA left factor x.A_e) */
+  E4B_STAGE_GATE_UP = 2,   /* grouped gate_up GEMM with dequant, LoRA delta, SwiGLU -> h */
+  E4B_STAGE_DOWN = 3,      /* grouped down GEMM with dequant -> y */
+  E4B_STAGE_COMBINE = 4    /* out[t] = sum_j w[t,j] * y[t,j] */
+};
+
+/*
+ * Runs one stage of e4b_moe_forward with the same arguments (for timing a
+ * single kernel).  Running E4B_STAGE_ROUTE .. E4B_STAGE_COMBINE in order on
+ * one stream and workspace is exactly e4b_moe_forward; a stage reads what the
+ * earlier stages left in the workspace.
+ */
+e4b_status e4b_moe_forward_stage(int32_t stage, const e4b_moe_desc* d, int32_t T, const uint16_t* x,
+                                 const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
+                                 const uint8_t* dn_codes, const void* dn_scales,
+                                 const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* out,
+                                 void* ws, size_t ws_bytes, e4b_stream stream);
+
+/* Intermediate buffers inside a forward workspace, for inspection. */
+enum {
+  E4B_WS_TOPK_IDS = 0,     /* int32 [T*k] */
+  E4B_WS_TOPK_W = 1,       /* fp32  [T*k] */
+  E4B_WS_EXPERT_OFFSETS = 2, /* int32 [E+1] */
+  E4B_WS_SORTED_SLOT = 3,  /* int32 [T*k] */
+  E4B_WS_X_SORTED = 4,     /* bf16  [T*k, H] */
+  E4B_WS_H = 5,            /* bf16  [T*k, I]  silu(gate)*up per routed row */
+  E4B_WS_Y = 6             /* fp32  [T*k, H]  down output per routed row */
+};
+
+/* Byte offset and size of one intermediate of e4b_moe_forward's workspace. */
+e4b_status e4b_moe_workspace_region(const e4b_moe_desc* d, int32_t T, int32_t region,
+                                    size_t* offset, size_t* bytes);
+
+/*
+ * Synchronises `stream`, then reads and clears the status word at the start
+ * of a workspace used by e4b_moe_forward or e4b_route.  Returns E4B_OK or the
+ * first device-side error recorded since the last call (E4B_ERR_TIMEOUT when
+ * a bounded wait ran out).
+ */
+e4b_status e4b_device_status(void* ws, e4b_stream stream);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one block that waits on
+ * a barrier nothing ever releases, with a limit of limit_ns nanoseconds (at
+ * most 10^9), then records E4B_ERR_TIMEOUT in the workspace status word and
+ * returns from the kernel.  Read the result with e4b_device_status().
+ */
+e4b_status e4b_debug_wait_timeout(uint32_t limit_ns, void* ws, size_t ws_bytes, e4b_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E4B_H */

@@ -85,8 +85,8 @@ def quantize_nf4(x):
         blk, a = blocks[b0:b0 + step], absmax[b0:b0 + step]
         nz = a != 0
         y = (blk[nz] / a[nz, None]).astype(np.float32)            # IEEE fp32 division
-        # code = number of midpoints strictly below y
-        codes[b0:b0 + step][nz] = np.sum(y[..., None] > mids, axis=-1).astype(np.uint8)
+        # code = number of midpoints strictly below y (a left-sided sorted search counts exactly those)
+        codes[b0:b0 + step][nz] = np.searchsorted(mids, y, side="left").astype(np.uint8)
     return pack_nf4(codes.reshape(-1)), absmax
 
 

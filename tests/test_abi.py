@@ -1,0 +1,76 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, its NF4 table equals the oracle's bit for bit, and host-side argument
+validation rejects bad calls before anything touches a GPU."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from bit_mixture_experts_top_b200 import e4b
+from oracle import nf4
+
+
+@pytest.fixture(scope="module")
+def L():
+    return e4b.lib()
+
+
+def test_library_exports_every_declared_function(L):
+    names = e4b.header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(e4b._SIGS), "binding and header disagree"
+
+
+def test_abi_version(L):
+    assert e4b.e4b_abi_version() == 1
+    assert L.e4b_status_string(4).decode().startswith("E4B_ERR_TIMEOUT")
+
+
+def test_library_nf4_table_equals_oracle_bit_for_bit():
+    got = e4b.e4b_nf4_codebook()
+    ref = nf4.nf4_codebook()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_format_calls_reject_bad_sizes_and_pointers(L):
+    assert L.e4b_dequant_mxfp4(None, None, 33, None, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_dequant_mxfp4(None, None, 32, None, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_dequant_mxfp4(None, None, 0, None, None) == e4b.E4B_OK           # empty: nothing to do
+    assert L.e4b_dequant_mxfp4(16, 16, 64, 24, None) == e4b.E4B_ERR_INVALID_ARG   # misaligned output
+    assert L.e4b_quantize_nf4(None, 96, None, None, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_quantize_nf4(None, 64, None, None, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_quantize_nf4(None, 0, None, None, None) == e4b.E4B_OK
+
+
+def test_route_validation(L):
+    assert L.e4b_route(None, 4, 8, 9, None, None, None, None, None, 0, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_route(None, 4, 300, 2, None, None, None, None, None, 0, None) == e4b.E4B_ERR_UNSUPPORTED
+    assert L.e4b_route(None, 4, 8, 2, None, None, 256, None, 256, 1 << 20, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_route_workspace_bytes(16, 8, 2) > 0
+    assert L.e4b_route_workspace_bytes(16, 8, 9) == 0
+
+
+def test_forward_validation_and_workspace(L):
+    d = e4b.make_desc(8, 256, 128, 2, "mxfp4")
+    ws = e4b.e4b_moe_workspace_bytes(d, 64)
+    # status + topk + offsets + histograms + slots + x_sorted + h + y, all 256-byte aligned
+    assert ws >= 64 * 2 * (256 * 2 + 128 * 2 + 256 * 4)
+    assert ws % 256 == 0
+    for bad in [e4b.make_desc(8, 250, 128, 2, "mxfp4"), e4b.make_desc(8, 256, 100, 2, "mxfp4"),
+                e4b.make_desc(8, 256, 128, 9, "mxfp4"), e4b.make_desc(300, 256, 128, 2, "nf4"),
+                e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=17),
+                e4b.make_desc(8, 256, 128, 2, "nf4", tokens_per_tile=48)]:
+        assert e4b.e4b_moe_workspace_bytes(bad, 64) == 0
+    # one-sided LoRA is refused before any launch
+    dl = e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=8, lora_scale=2.0)
+    st = L.e4b_moe_forward(ctypes.byref(dl), 4, None, None, None, None, None, None, 256, None, None, 256,
+                           1 << 30, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
+    # workspace too small
+    st = L.e4b_moe_forward(ctypes.byref(d), 64, 256, 256, 256, 256, 256, 256, None, None, 256, 256, 1024, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
+    off, nb = e4b.e4b_moe_workspace_region(d, 64, e4b.E4B_WS_H)
+    assert off % 256 == 0 and nb == 64 * 2 * 128 * 2 and off + nb <= ws
+    assert L.e4b_debug_wait_timeout(2_000_000_000, 256, 4096, None) == e4b.E4B_ERR_INVALID_ARG
