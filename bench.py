@@ -33,7 +33,7 @@ METRIC = "4-bit MoE layer tokens/s; decode weight GB/s vs HBM peak; prefill TFLO
 WORKLOAD = "qwen3_30b_a3b_nf4_decode"
 T_HEADLINE = 64
 L2_BYTES = 126 * 1000 * 1000
-KERNELS_PER_STEP = 6      # route_topk, route_rank, gather, gate_up GEMM, down GEMM, combine
+KERNELS_PER_STEP = 5      # route (top-k + rank, one block at T<=128), gather, gate_up GEMM, down GEMM, combine
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -227,21 +227,14 @@ def bench_e4b(args, world, rank, local):
     args_fwd = (lay.desc, T, x, lg, lay.gate_up.codes, lay.gate_up.scales, lay.down.codes, lay.down.scales,
                 lay.lora_A, lay.lora_B, out, ws)
 
-    def step(ev_g0=None, ev_g1=None, ev_d1=None):
-        for st in (e4b.E4B_STAGE_ROUTE, e4b.E4B_STAGE_GATHER):
-            e4b.e4b_moe_forward_stage(st, *args_fwd)
-        if ev_g0 is not None:
-            ev_g0.record()
-        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_GATE_UP, *args_fwd)
-        if ev_g1 is not None:
-            ev_g1.record()
-        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_DOWN, *args_fwd)
-        if ev_d1 is not None:
-            ev_d1.record()
-        e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_COMBINE, *args_fwd)
+    def forward():
+        e4b.e4b_moe_forward(*args_fwd)
+
+    def stage(st):
+        e4b.e4b_moe_forward_stage(st, *args_fwd)
 
     for _ in range(args.warmup):
-        step()
+        forward()
     torch.cuda.synchronize()
     if e4b.e4b_device_status(ws) != e4b.E4B_OK:
         raise RuntimeError("device status reported an error after warm-up")
@@ -252,28 +245,59 @@ def bench_e4b(args, world, rank, local):
     dn_bytes = touched * w.down_bytes_per_expert() + R * w.I * 2 + R * w.H * 4
     layer_weight_bytes = touched * (w.gate_up_bytes_per_expert() + w.down_bytes_per_expert())
 
+    # one step = one forward, replayed from a CUDA graph (the library's launches captured as-is)
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    g_fwd = capture(forward)
+    g_gu = capture(lambda: stage(e4b.E4B_STAGE_GATE_UP))
+    g_dn = capture(lambda: stage(e4b.E4B_STAGE_DOWN))
+    for _ in range(3):
+        g_fwd.replay()
+    torch.cuda.synchronize()
+
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(physical_gpu_index(local))
     barrier()
     torch.cuda.synchronize()
     sampler.start()
     t_start.record()
-    for i in range(K):
-        step(*evs[i])
+    for _ in range(K):
+        g_fwd.replay()
     t_end.record()
     torch.cuda.synchronize()
     clocks = sampler.summary()
     barrier()
     total_ms = t_start.elapsed_time(t_end)
-    gu_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
-    dn_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
     ms_per_step = max_over_ranks(total_ms / K)
-    gu_ms = max_over_ranks(gu_ms)
-    dn_ms = max_over_ranks(dn_ms)
+
+    def time_graph(g, n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        evs[0].record()
+        for i in range(n):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize()
+        return statistics.fmean(evs[i].elapsed_time(evs[i + 1]) for i in range(n))
+
+    # the dominant kernel, launch by launch (touched weights per launch exceed L2: no flush needed)
+    gu_ms = max_over_ranks(time_graph(g_gu, K))
+    dn_ms = max_over_ranks(time_graph(g_dn, K))
     if e4b.e4b_device_status(ws) != e4b.E4B_OK:
         raise RuntimeError("device status reported an error in the timed region")
+    del g_fwd, g_gu, g_dn
 
     # end to end through the public call with host buffers: H2D inputs, forward, D2H output, every step
     x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()

@@ -17,13 +17,15 @@
 // One persistent CTA per SM walks a tile list (expert, weight block, row
 // chunk); consecutive tiles share a weight block so its bytes are read from
 // HBM once and from L2 after.  Warp roles:
-//   warp 0      TMA producer: packed codes (64-byte swizzled boxes) into a raw
-//               ring, activation tiles (128-byte swizzled) into the B ring;
-//   warp 1      TMEM owner and single-thread UMMA issuer (kind::f16, M=128,
+//   warp 0      TMA producer of packed codes (64-byte swizzled boxes) into a
+//               raw ring; warms L2 with whole tiles (contiguous runs) ahead;
+//   warp 1      TMA producer of activation tiles (128-byte swizzled) into the
+//               B ring;
+//   warp 2      TMEM owner and single-thread UMMA issuer (kind::f16, M=128,
 //               N=BN, K=16, fp32 accumulators in TMEM, two buffers);
-//   warps 2-9   dequant: 4-bit codes + per-block scale -> bf16 written in the
+//   warps 3-10  dequant: 4-bit codes + per-block scale -> bf16 written in the
 //               128-byte-swizzled K-major layout the UMMA descriptor reads;
-//   warps 10-13 epilogue: tcgen05.ld, SwiGLU or fp32 store.
+//   warps 11-14 epilogue: tcgen05.ld, SwiGLU or fp32 store.
 // Every wait is bounded: on timeout the kernel records E4B_ERR_TIMEOUT, lets
 // copies and MMAs in flight land, frees its TMEM and returns.
 #include <cuda.h>
@@ -40,44 +42,54 @@ namespace e4b {
 namespace {
 
 constexpr int BM = 128;                      // weight rows per tile (UMMA M)
-constexpr int BK = 64;                       // K per MMA stage: one 128-byte swizzle row of bf16
+constexpr int ATOM_K = 64;                   // K per 128-byte swizzle row of bf16
+constexpr int A_ATOM_BYTES = BM * 128;       // one 128 x 64 bf16 swizzle atom column
 constexpr int RAW_K = 128;                   // K per packed-code stage
 constexpr int RAW_ROW_BYTES = RAW_K / 2;     // 64 bytes of codes per weight row
 constexpr int RAW_STAGE_BYTES = BM * RAW_ROW_BYTES;
-constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int LUT_BYTES = 32768;             // byte -> element-pair table, one copy per bank
 constexpr int NUM_DQ_WARPS = 8;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr int WARP_TMA = 0;
-constexpr int WARP_MMA = 1;
-constexpr int WARP_DQ0 = 2;
+constexpr int WARP_RAW = 0;                  // TMA producer of packed codes
+constexpr int WARP_ACT = 1;                  // TMA producer of activation tiles
+constexpr int WARP_MMA = 2;
+constexpr int WARP_DQ0 = 3;
 constexpr int WARP_EPI0 = WARP_DQ0 + NUM_DQ_WARPS;
 constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
 
+// Decode-sized tiles (BN <= 64) stage 128 K per MMA stage so each dequant
+// thread converts 64 elements per barrier round; prefill tiles (BN >= 128)
+// stage 64 K to leave shared memory for the wide B tiles.
 template <int BN>
 struct Cfg {
-  static constexpr int B_STAGE_BYTES = BN * BK * 2;
-  static constexpr int STAGES = BN >= 256 ? 3 : (BN >= 128 ? 4 : 6);
-  static constexpr int RAW_STAGES = 6;
+  static constexpr int BKS = BN <= 64 ? 128 : 64;
+  static constexpr int ATOMS = BKS / ATOM_K;
+  static constexpr int A_STAGE_BYTES = ATOMS * A_ATOM_BYTES;
+  static constexpr int B_ATOM_BYTES = BN * 128;
+  static constexpr int B_STAGE_BYTES = ATOMS * B_ATOM_BYTES;
+  static constexpr int STAGES = BN == 32 ? 2 : (BN == 64 ? 2 : (BN == 128 ? 4 : 3));
+  static constexpr int RAW_STAGES = BN == 32 ? 12 : (BN == 64 ? 10 : (BN == 128 ? 6 : 4));
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr int OFF_A = 0;
+  static constexpr int OFF_LUT = 0;
+  static constexpr int OFF_A = OFF_LUT + LUT_BYTES;
   static constexpr int OFF_B = OFF_A + STAGES * A_STAGE_BYTES;
   static constexpr int OFF_RAW = OFF_B + STAGES * B_STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_RAW + RAW_STAGES * RAW_STAGE_BYTES;
   static constexpr int NUM_BARS = 3 * STAGES + 2 * RAW_STAGES + 4;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_LUT = OFF_MISC + 16;
-  static constexpr int SMEM_BYTES = OFF_LUT + 64 + 1024;   // + slack to align the base to 1024
-  static_assert(B_STAGE_BYTES % 1024 == 0, "B stages must keep 1024-byte alignment");
-  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static constexpr int OFF_TAB = OFF_MISC + 16;              // chunk_off and expert_offsets, [E+1] each
+  static constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxExperts + 1) * 4 + 1024;   // + slack to align the base
+  static_assert(B_ATOM_BYTES % 1024 == 0, "B atoms must keep 1024-byte alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct Params {
   int32_t E, N, K, I;
   int32_t n_blocks;       // weight blocks per expert (mode 0: I/64 gate+up pairs; mode 1: ceil(N/128))
-  int32_t ksteps;         // K / 64
   int32_t lora_rank;      // 0 = none (mode 0 only)
+  const uint8_t* codes;   // packed stack [E, N, K/2] (for L2 warming)
   const void* scales;
   const uint16_t* lora_B; // [E, r, 2I]
   const int32_t* expert_offsets;
@@ -92,61 +104,101 @@ struct Tile {
   int e, nb, row0, rows;
 };
 
+// Tile lookup from the CTA's shared copies of chunk_off[E+1] and
+// expert_offsets[E+1] (tile order: expert, weight block, row chunk).
 template <int BN>
-__device__ __forceinline__ bool get_tile(const Params& p, int tile, int total, Tile& t) {
+__device__ __forceinline__ bool get_tile(const Params& p, const int32_t* s_chunk, const int32_t* s_off, int tile,
+                                         int total, Tile& t) {
   if (tile >= total) return false;
   int lo = 0, hi = p.E;                 // last e with chunk_off[e] * n_blocks <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(p.chunk_off + mid) * p.n_blocks <= tile) lo = mid; else hi = mid;
+    if (s_chunk[mid] * p.n_blocks <= tile) lo = mid; else hi = mid;
   }
-  const int c0 = __ldg(p.chunk_off + lo);
-  const int nch = __ldg(p.chunk_off + lo + 1) - c0;
+  const int c0 = s_chunk[lo];
+  const int nch = s_chunk[lo + 1] - c0;
   const int local = tile - c0 * p.n_blocks;
   t.e = lo;
   t.nb = local / nch;
   const int chunk = local - t.nb * nch;
-  const int off = __ldg(p.expert_offsets + lo);
-  t.row0 = off + chunk * BN;
-  t.rows = min(BN, __ldg(p.expert_offsets + lo + 1) - t.row0);
+  t.row0 = s_off[lo] + chunk * BN;
+  t.rows = min(BN, s_off[lo + 1] - t.row0);
   return true;
+}
+
+// Row of the weight stack behind A-tile row `prow` (mode 0 pairs gate and up
+// rows: within each 32-row group, rows 0..15 are gate features and 16..31 the
+// matching up features) and its row in the raw code tile.
+template <int MODE>
+__device__ __forceinline__ void tile_row(const Params& p, int nb, int prow, int& wrow, int& raw_row) {
+  if (MODE == 0) {
+    const int g = prow >> 5, wi = prow & 31;
+    const int f = 64 * nb + 16 * g + (wi & 15);
+    raw_row = (wi < 16 ? 0 : 64) + 16 * g + (wi & 15);
+    wrow = (wi < 16) ? f : p.I + f;
+  } else {
+    raw_row = prow;
+    wrow = BM * nb + prow;
+  }
 }
 
 __device__ __forceinline__ float e2m1_to_f32(uint32_t nib) {
   return __uint_as_float(((nib & 8u) << 28) | ((nib & 7u) << 22)) * 0x1p126f;
 }
 
-__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
-  return __uint_as_float(s == 0u ? 0x00400000u : (s == 255u ? 0x7FC00000u : (s << 23)));
+// bf16x2 of the E8M0 scale 2^(s-127) in both halves (s = 0: bf16 subnormal, 255: NaN).
+__device__ __forceinline__ uint32_t e8m0_to_bf16x2(uint32_t s) {
+  const uint32_t b = s == 0u ? 0x0040u : (s == 255u ? 0x7FC0u : (s << 7));
+  return b | (b << 16);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+// NF4: one code byte -> two bf16 (element 2j from the high nibble in the low
+// half).  The LUT holds fp32 level pairs; the fp32 products round once.
+__device__ __forceinline__ uint32_t nf4_pair(uint32_t addr, uint64_t a2) {
+  uint32_t r;
+  asm("{\n\t.reg .b64 t;\n\t.reg .f32 lo, hi;\n\t"
+      "ld.shared.b64 t, [%1];\n\t"
+      "mul.rn.f32x2 t, t, %2;\n\t"
+      "mov.b64 {lo, hi}, t;\n\t"
+      "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+      : "=r"(r)
+      : "r"(addr), "l"(a2));
+  return r;
 }
 
-// 16 code bytes (32 elements, one scale) -> 4 x 16 bytes of bf16 in element order.
+// MXFP4: one code byte -> two bf16 (element 2j from the low nibble in the low
+// half).  The LUT holds exact bf16 pairs; the power-of-two scale keeps them exact.
+__device__ __forceinline__ uint32_t mx_pair(uint32_t addr, uint32_t s2) {
+  uint32_t r;
+  asm("{\n\t.reg .b32 t;\n\t"
+      "ld.shared.b32 t, [%1];\n\t"
+      "mul.rn.bf16x2 %0, t, %2;\n\t}"
+      : "=r"(r)
+      : "r"(addr), "r"(s2));
+  return r;
+}
+
+// 16 code bytes (32 elements sharing one scale) -> 4 x 16 bytes of bf16.
+// lut_l already includes this lane's table copy; scale is the fp32 absmax
+// (NF4) or the bf16x2 E8M0 scale (MXFP4).
 template <int FMT>
-__device__ __forceinline__ void dequant32(const uint4 q, float sc, const float* lut, uint4 (&o)[4]) {
+__device__ __forceinline__ void dequant32(const uint4 q, uint32_t lut_l, uint64_t a2, uint32_t s2, uint4 (&o)[4]) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     uint32_t r[4];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const uint32_t byte = (w[i] >> (8 * b)) & 0xFFu;
-      float f0, f1;
-      if (FMT == E4B_NF4) {           // element 2j in the high nibble
-        f0 = lut[byte >> 4] * sc;
-        f1 = lut[byte & 0xFu] * sc;
-      } else {                        // MXFP4: element 2j in the low nibble
-        f0 = e2m1_to_f32(byte & 0xFu) * sc;
-        f1 = e2m1_to_f32(byte >> 4) * sc;
-      }
-      r[b] = pack_bf16x2(f0, f1);
+      const uint32_t addr = lut_l + (((w[i] >> (8 * b)) & 0xFFu) << 7);
+      r[b] = FMT == E4B_NF4 ? nf4_pair(addr, a2) : mx_pair(addr, s2);
     }
     o[i] = make_uint4(r[0], r[1], r[2], r[3]);
   }
+}
+
+__device__ __forceinline__ uint64_t dup_f32(float a) {
+  const uint64_t u = __float_as_uint(a);
+  return u | (u << 32);
 }
 
 template <int BN, int FMT, int MODE>
@@ -156,6 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* sLut = smem + C::OFF_LUT;
   uint8_t* sA = smem + C::OFF_A;
   uint8_t* sB = smem + C::OFF_B;
   uint8_t* sRaw = smem + C::OFF_RAW;
@@ -169,7 +222,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int32_t* s_abort = reinterpret_cast<int32_t*>(smem + C::OFF_MISC + 8);
-  float* s_lut = reinterpret_cast<float*>(smem + C::OFF_LUT);
+  int32_t* s_chunk = reinterpret_cast<int32_t*>(smem + C::OFF_TAB);
+  int32_t* s_off = s_chunk + (kMaxExperts + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -189,8 +243,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     *s_abort = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 16) s_lut[threadIdx.x] = p.lut[threadIdx.x];
-  if (warp == WARP_TMA && lane == 0) {
+  // Byte -> element-pair tables, replicated so that every lane of a warp reads
+  // its own bank: NF4 fp32 pairs (16 copies of 8 bytes per byte value), MXFP4
+  // bf16 pairs (32 copies of 4 bytes).
+  if (FMT == E4B_NF4) {
+    float2* lut = reinterpret_cast<float2*>(sLut);
+    for (int i = threadIdx.x; i < 256 * 16; i += NUM_THREADS) {
+      const int b = i >> 4;
+      lut[i] = make_float2(p.lut[b >> 4], p.lut[b & 15]);
+    }
+  } else {
+    uint32_t* lut = reinterpret_cast<uint32_t*>(sLut);
+    for (int i = threadIdx.x; i < 256 * 32; i += NUM_THREADS) {
+      const int b = i >> 5;
+      __nv_bfloat162 v = __floats2bfloat162_rn(e2m1_to_f32(b & 15), e2m1_to_f32(b >> 4));
+      lut[i] = *reinterpret_cast<uint32_t*>(&v);
+    }
+  }
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
+    s_chunk[i] = __ldg(p.chunk_off + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
+  }
+  if (warp == WARP_RAW && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_act);
     if (MODE == 0 && p.lora_rank > 0) tma_prefetch_desc(&tm_xa);
@@ -205,49 +279,90 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *s_tmem;
 
   const WaitCtx wctx{s_abort, p.status, p.wait_limit_ns};
-  const int total = __ldg(p.chunk_off + p.E) * p.n_blocks;
+  const int total = s_chunk[p.E] * p.n_blocks;
   const bool lora = (MODE == 0) && p.lora_rank > 0;
-  const int nsteps = p.ksteps + (lora ? 1 : 0);
+  const int raw_steps = (p.K + RAW_K - 1) / RAW_K;
+  const int mma_steps = (p.K + C::BKS - 1) / C::BKS;   // K stages per tile (before the LoRA step)
+  const int nsteps = mma_steps + (lora ? 1 : 0);
 
-  if (warp == WARP_TMA) {
-    // ------------------------------------------------------------ producer
+  if (warp == WARP_RAW) {
+    // ------------------------------------------------------------ packed-code producer
     if (lane == 0) {
-      int stage = 0, rstage = 0;
-      uint32_t phase = 0, rphase = 0;
-      uint32_t armed_b = 0, armed_r = 0, par_b = 0, par_r = 0;   // per-stage "armed" bit and parity
+      int rstage = 0;
+      uint32_t rphase = 0, armed_r = 0, par_r = 0;   // per-stage "armed" bit and parity
       bool ok = true;
+      // Each tile's packed codes are one (down) or two (gate_up) contiguous runs
+      // of the stack, and so are its scale rows: warm L2 with whole runs, one
+      // tile ahead, so HBM streams them sequentially and the per-stage boxes hit L2.
+      auto warm_tile = [&](int tile_id) {
+        Tile wt;
+        if (!get_tile<BN>(p, s_chunk, s_off, tile_id, total, wt)) return;
+        const int nrun = MODE == 0 ? 2 : 1;
+        for (int run = 0; run < nrun; ++run) {
+          const int row0 = MODE == 0 ? (run == 0 ? 64 * wt.nb : p.I + 64 * wt.nb) : BM * wt.nb;
+          const int nrows = MODE == 0 ? 64 : min(BM, p.N - row0);
+          const int64_t grow = static_cast<int64_t>(wt.e) * p.N + row0;
+          bulk_prefetch_l2(p.codes + grow * (p.K / 2), static_cast<uint32_t>(nrows) * (p.K / 2));
+          const int sbytes = FMT == E4B_NF4 ? p.K / 16 : p.K / 32;     // scale bytes per row
+          const uint32_t sz = (static_cast<uint32_t>(nrows) * sbytes) & ~15u;
+          const uint8_t* sp = reinterpret_cast<const uint8_t*>(p.scales) + grow * sbytes;
+          const uint8_t* spa = reinterpret_cast<const uint8_t*>(reinterpret_cast<uintptr_t>(sp) & ~uintptr_t(15));
+          if (sz) bulk_prefetch_l2(spa, sz);
+        }
+      };
+      warm_tile(blockIdx.x);
+      warm_tile(blockIdx.x + gridDim.x);
       Tile t;
-      for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x) {
-        for (int ks = 0; ks < nsteps; ++ks) {
-          if (ks < p.ksteps && (ks & 1) == 0) {
-            if (!mbar_wait(&raw_empty[rstage], rphase ^ 1u, wctx, 101)) { ok = false; break; }
-            mbar_arrive_expect_tx(&raw_full[rstage], RAW_STAGE_BYTES);
-            uint8_t* dst = sRaw + rstage * RAW_STAGE_BYTES;
-            const int x = ks * (BK / 2);
-            if (MODE == 0) {
-              tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + 64 * t.nb);
-              tma_load_2d(dst + 64 * RAW_ROW_BYTES, &tm_codes, &raw_full[rstage], x, t.e * p.N + p.I + 64 * t.nb);
-            } else {
-              tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + BM * t.nb);
-            }
-            armed_r |= 1u << rstage;
-            par_r = (par_r & ~(1u << rstage)) | (rphase << rstage);
-            if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
+      for (int tile = blockIdx.x; ok && get_tile<BN>(p, s_chunk, s_off, tile, total, t); tile += gridDim.x) {
+        warm_tile(tile + 2 * gridDim.x);
+        for (int r = 0; r < raw_steps; ++r) {
+          if (!mbar_wait(&raw_empty[rstage], rphase ^ 1u, wctx, 101)) { ok = false; break; }
+          mbar_arrive_expect_tx(&raw_full[rstage], RAW_STAGE_BYTES);
+          uint8_t* dst = sRaw + rstage * RAW_STAGE_BYTES;
+          const int x = r * RAW_ROW_BYTES;
+          if (MODE == 0) {
+            tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + 64 * t.nb);
+            tma_load_2d(dst + 64 * RAW_ROW_BYTES, &tm_codes, &raw_full[rstage], x, t.e * p.N + p.I + 64 * t.nb);
+          } else {
+            tma_load_2d(dst, &tm_codes, &raw_full[rstage], x, t.e * p.N + BM * t.nb);
           }
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 102)) { ok = false; break; }
-          mbar_arrive_expect_tx(&b_full[stage], C::B_STAGE_BYTES);
-          if (ks < p.ksteps)
-            tma_load_2d(sB + stage * C::B_STAGE_BYTES, &tm_act, &b_full[stage], ks * BK, t.row0);
-          else
-            tma_load_2d(sB + stage * C::B_STAGE_BYTES, &tm_xa, &b_full[stage], 0, t.row0);
-          armed_b |= 1u << stage;
-          par_b = (par_b & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          armed_r |= 1u << rstage;
+          par_r = (par_r & ~(1u << rstage)) | (rphase << rstage);
+          if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
         }
       }
       if (!ok) {   // let every issued copy land before the CTA's shared memory is released
         for (int s = 0; s < C::RAW_STAGES; ++s)
           if (armed_r & (1u << s)) mbar_drain(&raw_full[s], (par_r >> s) & 1u, kDrainNs);
+      }
+    }
+  } else if (warp == WARP_ACT) {
+    // ------------------------------------------------------------ activation producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, armed_b = 0, par_b = 0;
+      bool ok = true;
+      Tile t;
+      for (int tile = blockIdx.x; ok && get_tile<BN>(p, s_chunk, s_off, tile, total, t); tile += gridDim.x) {
+        for (int ks = 0; ks < nsteps; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 102)) { ok = false; break; }
+          if (ks < mma_steps) {
+            const int k0 = ks * C::BKS;
+            const int natoms = min(C::ATOMS, (p.K - k0) / ATOM_K);
+            mbar_arrive_expect_tx(&b_full[stage], natoms * C::B_ATOM_BYTES);
+            for (int a = 0; a < natoms; ++a)
+              tma_load_2d(sB + stage * C::B_STAGE_BYTES + a * C::B_ATOM_BYTES, &tm_act, &b_full[stage],
+                          k0 + a * ATOM_K, t.row0);
+          } else {                                   // LoRA step: the xa tile
+            mbar_arrive_expect_tx(&b_full[stage], C::B_ATOM_BYTES);
+            tma_load_2d(sB + stage * C::B_STAGE_BYTES, &tm_xa, &b_full[stage], 0, t.row0);
+          }
+          armed_b |= 1u << stage;
+          par_b = (par_b & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
         for (int s = 0; s < C::STAGES; ++s)
           if (armed_b & (1u << s)) mbar_drain(&b_full[s], (par_b >> s) & 1u, kDrainNs);
       }
@@ -262,7 +377,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint64_t* last_bar = nullptr;
       uint32_t last_par = 0;
       Tile t;
-      for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x, ++it) {
+      for (int tile = blockIdx.x; ok && get_tile<BN>(p, s_chunk, s_off, tile, total, t); tile += gridDim.x, ++it) {
         const int buf = it & 1;
         const uint32_t aphase = (it >> 1) & 1;
         if (!mbar_wait(&acc_empty[buf], aphase ^ 1u, wctx, 201)) { ok = false; break; }
@@ -272,12 +387,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&a_full[stage], phase, wctx, 202)) { ok = false; break; }
           if (!mbar_wait(&b_full[stage], phase, wctx, 203)) { ok = false; break; }
           tc_fence_after_sync();
-          const uint32_t a0 = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t a0 = smem_u32(sA + stage * C::A_STAGE_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_STAGE_BYTES);
-          const int nk = ks < p.ksteps ? BK / 16 : 1;       // the LoRA step is one K=16 MMA
-          for (int kk = 0; kk < nk; ++kk)
-            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc,
+          // K16 steps: 4 per valid atom; the LoRA step is a single K=16 MMA
+          const int nk = ks < mma_steps ? 4 * min(C::ATOMS, (p.K - ks * C::BKS) / ATOM_K) : 1;
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t ao = (kk >> 2) * A_ATOM_BYTES + (kk & 3) * 32;
+            const uint32_t bo = (kk >> 2) * C::B_ATOM_BYTES + (kk & 3) * 32;
+            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + ao), smem_desc_sw128(b0 + bo), idesc,
                          (ks > 0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit(&empty[stage]);
           issued = true;
           last_bar = &empty[stage];
@@ -295,49 +414,98 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ dequant
     const int dt = threadIdx.x - WARP_DQ0 * 32;   // 0..255
     const int prow = dt & (BM - 1);               // A-tile row written by this thread
-    const int half = dt >> 7;                     // 32-element half of each 64-wide K stage
+    const int half = dt >> 7;                     // BKS 128: atom; BKS 64: 32-element half of the atom
+    const uint32_t lut_l =
+        smem_u32(sLut) + (FMT == E4B_NF4 ? static_cast<uint32_t>(lane & 15) * 8u : static_cast<uint32_t>(lane) * 4u);
+    const int kb64 = p.K / 64, kb32 = p.K / 32;
     int stage = 0, rstage = 0;
     uint32_t phase = 0, rphase = 0;
     bool ok = true;
     Tile t;
-    for (int tile = blockIdx.x; ok && get_tile<BN>(p, tile, total, t); tile += gridDim.x) {
-      int raw_row, wrow;
-      if (MODE == 0) {                              // rows 32g..32g+15 gate, 32g+16..32g+31 up
-        const int g = prow >> 5, wi = prow & 31;
-        const int f = 64 * t.nb + 16 * g + (wi & 15);
-        raw_row = (wi < 16 ? 0 : 64) + 16 * g + (wi & 15);
-        wrow = (wi < 16) ? f : p.I + f;
-      } else {
-        raw_row = prow;
-        wrow = BM * t.nb + prow;
-      }
+    for (int tile = blockIdx.x; ok && get_tile<BN>(p, s_chunk, s_off, tile, total, t); tile += gridDim.x) {
+      int wrow, raw_row;
+      tile_row<MODE>(p, t.nb, prow, wrow, raw_row);
       const int64_t grow = static_cast<int64_t>(t.e) * p.N + min(wrow, p.N - 1);
-      const float* sc_nf4 = reinterpret_cast<const float*>(p.scales) + grow * (p.K / 64);
-      const uint8_t* sc_mx = reinterpret_cast<const uint8_t*>(p.scales) + grow * (p.K / 32) + half;
-      auto load_scale = [&](int ks) -> float {
-        return FMT == E4B_NF4 ? __ldg(sc_nf4 + ks) : e8m0_to_f32(__ldg(sc_mx + 2 * ks));
-      };
-      float sc_next = load_scale(0);
-      for (int ks = 0; ks < p.ksteps; ++ks) {
-        const float sc = sc_next;
-        if (ks + 1 < p.ksteps) sc_next = load_scale(ks + 1);
-        if ((ks & 1) == 0 && !mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
-        if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
-        const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
-        const uint4 q = *reinterpret_cast<const uint4*>(
-            raw + swizzled_offset(raw_row, (ks & 1) * 2 + half, RAW_ROW_BYTES));
-        uint4 o[4];
-        dequant32<FMT>(q, sc, s_lut, o);
-        uint8_t* a = sA + stage * A_STAGE_BYTES;
+      const float* sc_nf4 = reinterpret_cast<const float*>(p.scales) + grow * kb64;
+      const uint8_t* sc_mx = reinterpret_cast<const uint8_t*>(p.scales) + grow * kb32;
+      if (C::BKS == 128) {
+        // each thread: 64 elements of its row per stage (atom `half`)
+        // scales of this thread's 64 elements: NF4 one absmax, MXFP4 two E8M0 (one per 32)
+        auto load_scale = [&](int r, uint64_t& a2, uint32_t& s2a, uint32_t& s2b) {
+          const int blk = 2 * r + half;                     // 64-element block along K
+          if (blk >= kb64) return;                          // ragged tail: nothing to decode
+          if (FMT == E4B_NF4) {
+            a2 = dup_f32(__ldg(sc_nf4 + blk));
+          } else {
+            const uint32_t v = __ldg(reinterpret_cast<const uint16_t*>(sc_mx + 2 * blk));
+            s2a = e8m0_to_bf16x2(v & 0xFFu);
+            s2b = e8m0_to_bf16x2(v >> 8);
+          }
+        };
+        uint64_t a2n = 0;
+        uint32_t san = 0, sbn = 0;
+        load_scale(0, a2n, san, sbn);
+        for (int r = 0; r < raw_steps; ++r) {
+          const uint64_t a2 = a2n;
+          const uint32_t sa = san, sb = sbn;
+          if (r + 1 < raw_steps) load_scale(r + 1, a2n, san, sbn);
+          if (!mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
+          if (r * RAW_K + half * ATOM_K < p.K) {
+            const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
+            uint8_t* a = sA + stage * C::A_STAGE_BYTES + half * A_ATOM_BYTES;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[stage]);
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-        if ((ks & 1) == 1 || ks + 1 == p.ksteps) {
-          if (lane == 0) mbar_arrive(&raw_empty[rstage]);
+            for (int c = 0; c < 2; ++c) {
+              const uint4 q =
+                  *reinterpret_cast<const uint4*>(raw + swizzled_offset(raw_row, half * 2 + c, RAW_ROW_BYTES));
+              uint4 o[4];
+              dequant32<FMT>(q, lut_l, a2, c == 0 ? sa : sb, o);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4*>(a + swizzled_offset(prow, c * 4 + i, 128)) = o[i];
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&a_full[stage]);
+            mbar_arrive(&raw_empty[rstage]);
+          }
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
           if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
+        }
+      } else {
+        // each thread: 32 elements (half of one 64-wide atom row) per MMA stage
+        auto load_scale = [&](int ks, uint64_t& a2, uint32_t& s2) {
+          if (FMT == E4B_NF4) a2 = dup_f32(__ldg(sc_nf4 + ks));
+          else s2 = e8m0_to_bf16x2(__ldg(sc_mx + 2 * ks + half));
+        };
+        const int ksteps = p.K / ATOM_K;
+        uint64_t a2n = 0;
+        uint32_t s2n = 0;
+        load_scale(0, a2n, s2n);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          const uint64_t a2 = a2n;
+          const uint32_t s2 = s2n;
+          if (ks + 1 < ksteps) load_scale(ks + 1, a2n, s2n);
+          if ((ks & 1) == 0 && !mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
+          const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
+          const uint4 q = *reinterpret_cast<const uint4*>(
+              raw + swizzled_offset(raw_row, (ks & 1) * 2 + half, RAW_ROW_BYTES));
+          uint4 o[4];
+          dequant32<FMT>(q, lut_l, a2, s2, o);
+          uint8_t* a = sA + stage * C::A_STAGE_BYTES;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if ((ks & 1) == 1 || ks + 1 == ksteps) {
+            if (lane == 0) mbar_arrive(&raw_empty[rstage]);
+            if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
+          }
         }
       }
       if (!ok) break;
@@ -352,7 +520,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t hi = (2 * j + 1 < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * j + 1) * 2 * p.I) : 0u;
             v[j] = lo | (hi << 16);
           }
-          uint8_t* a = sA + stage * A_STAGE_BYTES;
+          uint8_t* a = sA + stage * C::A_STAGE_BYTES;
           *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 0, 128)) = make_uint4(v[0], v[1], v[2], v[3]);
           *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 1, 128)) = make_uint4(v[4], v[5], v[6], v[7]);
         }
@@ -367,10 +535,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;                        // TMEM lanes 32q..32q+31
     int it = 0;
     Tile t;
-    for (int tile = blockIdx.x; get_tile<BN>(p, tile, total, t); tile += gridDim.x, ++it) {
+    for (int tile = blockIdx.x; get_tile<BN>(p, s_chunk, s_off, tile, total, t); tile += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t aphase = (it >> 1) & 1;
-      if (!mbar_wait(&acc_full[buf], aphase, wctx, 401)) break;
+      if (!mbar_wait_sleep(&acc_full[buf], aphase, wctx, 401, 256)) break;
       tc_fence_after_sync();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
       for (int c0 = 0; c0 < BN && c0 < t.rows; c0 += 16) {
@@ -479,12 +647,12 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   if (!encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, RAW_ROW_BYTES,
                  g.mode == 0 ? 64 : BM, CU_TENSOR_MAP_SWIZZLE_64B))
     return E4B_ERR_CUDA;
-  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, BK, BN,
+  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, ATOM_K, BN,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return E4B_ERR_CUDA;
   const bool lora = g.mode == 0 && g.lora_rank > 0;
   if (lora) {
-    if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.xa, 64, g.R, 128, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.xa, 64, g.R, 128, ATOM_K, BN, CU_TENSOR_MAP_SWIZZLE_128B))
       return E4B_ERR_CUDA;
   } else {
     tx = ta;
@@ -495,8 +663,8 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.K = g.K;
   prm.I = g.I;
   prm.n_blocks = g.mode == 0 ? g.I / 64 : (g.N + BM - 1) / BM;
-  prm.ksteps = g.K / BK;
   prm.lora_rank = lora ? g.lora_rank : 0;
+  prm.codes = g.codes;
   prm.scales = g.scales;
   prm.lora_B = g.lora_B;
   prm.expert_offsets = g.expert_offsets;

@@ -36,12 +36,66 @@ __device__ __forceinline__ uint32_t route_key(uint16_t bits, int e) {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
+// Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
+// slots of the block with the same expert).  Each warp owns a contiguous
+// segment; per-warp histograms are scanned across warps first.
+__device__ __forceinline__ void rank_block(int b, const int32_t* __restrict__ topk_ids, int T, int E, int k,
+                                           const int32_t* block_base, int32_t* __restrict__ sorted_slot,
+                                           int32_t* __restrict__ slot_pos, int32_t (*s_wc)[kMaxExperts]) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t s0 = static_cast<int64_t>(b) * kRouteTokensPerBlock * k;
+  const int64_t s1 = min(static_cast<int64_t>(T), static_cast<int64_t>(b + 1) * kRouteTokensPerBlock) * k;
+  const int64_t n = s1 - s0;
+  const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t w0 = s0 + warp * seg, w1 = min(s1, w0 + seg);
+  for (int i = tid; i < kWarps * kMaxExperts; i += kThreads) (&s_wc[0][0])[i] = 0;
+  __syncthreads();
+  for (int64_t s = w0 + lane; s < w1; s += 32) atomicAdd(&s_wc[warp][topk_ids[s]], 1);
+  __syncthreads();
+  for (int e = tid; e < E; e += kThreads) {
+    int32_t run = __ldcg(block_base + static_cast<int64_t>(b) * E + e);
+    for (int w = 0; w < kWarps; ++w) {
+      const int32_t c = s_wc[w][e];
+      s_wc[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t c0 = w0; c0 < w1; c0 += 32) {
+    const int64_t s = c0 + lane;
+    const bool valid = s < w1;
+    const int id = valid ? topk_ids[s] : (kMaxExperts + lane);   // invalid lanes never match
+    const uint32_t peers = __match_any_sync(kFull, id);
+    const int rank = __popc(peers & lt);
+    int32_t pos = 0;
+    if (valid) pos = s_wc[warp][id] + rank;
+    __syncwarp();
+    if (valid && rank == __popc(peers) - 1) s_wc[warp][id] += __popc(peers);
+    __syncwarp();
+    if (valid) {
+      sorted_slot[pos] = static_cast<int32_t>(s);
+      slot_pos[s] = pos;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __restrict__ topk_ids, int T, int E,
+                                                              int k, const int32_t* __restrict__ block_base,
+                                                              int32_t* __restrict__ sorted_slot,
+                                                              int32_t* __restrict__ slot_pos) {
+  __shared__ int32_t s_wc[kWarps][kMaxExperts];
+  rank_block(blockIdx.x, topk_ids, T, E, k, block_base, sorted_slot, slot_pos, s_wc);
+}
+
 __global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E, int k,
                                                               int tokens_per_tile, int nblk,
                                                               int32_t* __restrict__ topk_ids,
                                                               float* __restrict__ topk_w, int32_t* block_counts,
                                                               uint32_t* done_counter, int32_t* expert_offsets,
-                                                              int32_t* chunk_off) {
+                                                              int32_t* chunk_off, int32_t* __restrict__ sorted_slot,
+                                                              int32_t* __restrict__ slot_pos) {
+  __shared__ int32_t s_wc[kWarps][kMaxExperts];
   __shared__ int32_t s_cnt[kMaxExperts];
   __shared__ int32_t s_tot[kMaxExperts + 1];
   __shared__ bool s_last;
@@ -130,51 +184,10 @@ __global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __
       run += c;
     }
   }
-}
-
-// Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
-// slots of the block with the same expert).  Each warp owns a contiguous
-// segment; per-warp histograms are scanned across warps first.
-__global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __restrict__ topk_ids, int T, int E,
-                                                              int k, const int32_t* __restrict__ block_base,
-                                                              int32_t* __restrict__ sorted_slot,
-                                                              int32_t* __restrict__ slot_pos) {
-  __shared__ int32_t s_wc[kWarps][kMaxExperts];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock * k;
-  const int64_t s1 = min(static_cast<int64_t>(T), static_cast<int64_t>(blockIdx.x + 1) * kRouteTokensPerBlock) * k;
-  const int64_t n = s1 - s0;
-  const int64_t seg = ((n + kWarps - 1) / kWarps + 31) / 32 * 32;
-  const int64_t w0 = s0 + warp * seg, w1 = min(s1, w0 + seg);
-  for (int i = tid; i < kWarps * kMaxExperts; i += kThreads) (&s_wc[0][0])[i] = 0;
-  __syncthreads();
-  for (int64_t s = w0 + lane; s < w1; s += 32) atomicAdd(&s_wc[warp][topk_ids[s]], 1);
-  __syncthreads();
-  for (int e = tid; e < E; e += kThreads) {
-    int32_t run = block_base[static_cast<int64_t>(blockIdx.x) * E + e];
-    for (int w = 0; w < kWarps; ++w) {
-      const int32_t c = s_wc[w][e];
-      s_wc[w][e] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int64_t c0 = w0; c0 < w1; c0 += 32) {
-    const int64_t s = c0 + lane;
-    const bool valid = s < w1;
-    const int id = valid ? topk_ids[s] : (kMaxExperts + lane);   // invalid lanes never match
-    const uint32_t peers = __match_any_sync(kFull, id);
-    const int rank = __popc(peers & lt);
-    int32_t pos = 0;
-    if (valid) pos = s_wc[warp][id] + rank;
-    __syncwarp();
-    if (valid && rank == __popc(peers) - 1) s_wc[warp][id] += __popc(peers);
-    __syncwarp();
-    if (valid) {
-      sorted_slot[pos] = static_cast<int32_t>(s);
-      slot_pos[s] = pos;
-    }
+  if (nblk == 1) {          // a single routing block also ranks its slots: one launch for small batches
+    __threadfence_block();
+    __syncthreads();
+    rank_block(0, topk_ids, T, E, k, block_counts, sorted_slot, slot_pos, s_wc);
   }
 }
 
@@ -198,6 +211,8 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __rest
 #pragma unroll
   for (int j = 0; j < kMaxLoraRank; ++j) acc[j] = 0.0f;
   const uint16_t* Ae = lora_A ? lora_A + static_cast<int64_t>(topk_ids[slot]) * H * rank : nullptr;
+  const bool vec8 = Ae && (rank == 8 || rank == 16) &&            // A rows are whole 16-byte vectors
+                    (reinterpret_cast<uintptr_t>(lora_A) & 15u) == 0;
   for (int v = lane; v < nvec; v += 32) {
     const uint4 q = __ldg(src + v);
     dst[v] = q;
@@ -207,9 +222,23 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __rest
       for (int i = 0; i < 8; ++i) {
         const float xv = bf16_bits_to_f32(static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1))));
         const uint16_t* arow = Ae + static_cast<int64_t>(v * 8 + i) * rank;
+        if (vec8) {
 #pragma unroll
-        for (int j = 0; j < kMaxLoraRank; ++j)
-          if (j < rank) acc[j] = fmaf(xv, bf16_bits_to_f32(__ldg(arow + j)), acc[j]);
+          for (int h = 0; h < kMaxLoraRank / 8; ++h) {
+            if (h * 8 < rank) {
+              const uint4 a = __ldg(reinterpret_cast<const uint4*>(arow) + h);
+              const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                acc[h * 8 + j] = fmaf(xv, bf16_bits_to_f32(static_cast<uint16_t>(aw[j >> 1] >> (16 * (j & 1)))),
+                                      acc[h * 8 + j]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kMaxLoraRank; ++j)
+            if (j < rank) acc[j] = fmaf(xv, bf16_bits_to_f32(__ldg(arow + j)), acc[j]);
+        }
       }
     }
   }
@@ -265,9 +294,10 @@ cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k
   }
   const int nblk = route_blocks(T);
   route_topk_kernel<<<nblk, kThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
-                                               b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off);
+                                               b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off,
+                                               b.sorted_slot, b.slot_pos);
   cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  if (err != cudaSuccess || nblk == 1) return err;
   route_rank_kernel<<<nblk, kThreads, 0, s>>>(b.topk_ids, T, E, k, b.block_counts, b.sorted_slot, b.slot_pos);
   return cudaGetLastError();
 }
