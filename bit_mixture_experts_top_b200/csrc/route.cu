@@ -321,3 +321,78 @@ cudaError_t launch_combine(const float* y, const float* topk_w, const int32_t* s
 }
 
 }  // namespace e4b
+
+// ---------------------------------------------------------------------------
+// Routing for callers that cannot allocate device memory.
+//
+// Some callers have no way to hand the library a workspace: a host runtime
+// that owns every byte of device memory through its own pool and forbids
+// cudaMalloc once it has started, or a latency-critical serving loop where an
+// allocation could synchronise the device.  e4b_route_noalloc runs the same
+// routing kernels as e4b_route but keeps their scratch (status word, per-block
+// histograms, slot positions) in one file-scope device array of fixed size
+// that every GPU loading the library holds until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace e4b {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;     // 1 MiB per device
+static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
+
+// Device addresses of g_route_scratch, looked up once per device.  In host
+// code the array's name is only a host-side handle: the address the kernels
+// need comes from cudaGetSymbolAddress with that device current.
+uint8_t* g_route_scratch_addr[64] = {};
+std::mutex g_route_scratch_mu;
+
+e4b_status route_scratch_address(uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return E4B_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+  if (!g_route_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return E4B_ERR_CUDA;
+    g_route_scratch_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_route_scratch_addr[dev];
+  return E4B_OK;
+}
+
+}  // namespace
+}  // namespace e4b
+
+extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_ids,
+                                        float* topk_w, int32_t* expert_offsets, int32_t* sorted_slot,
+                                        e4b_stream stream) {
+  using namespace e4b;
+  if (T < 0 || E < 1 || k < 1 || k > E) return E4B_ERR_INVALID_ARG;
+  if (E > kMaxExperts || k > kMaxTopK) return E4B_ERR_UNSUPPORTED;
+  if (!expert_offsets) return E4B_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_ids || !topk_w || !sorted_slot)) return E4B_ERR_INVALID_ARG;
+  // scratch layout: status word + done counter, per-block histograms, slot positions
+  const size_t nblk = static_cast<size_t>(route_blocks(T) > 0 ? route_blocks(T) : 1);
+  const size_t off_counts = align_up(kStatusBytes);
+  const size_t off_pos = off_counts + align_up(nblk * static_cast<size_t>(E) * 4);
+  const size_t need = off_pos + align_up(static_cast<size_t>(T) * k * 4);
+  if (need > kNoAllocScratchBytes) return E4B_ERR_UNSUPPORTED;   // beyond the fixed scratch size
+  uint8_t* scratch = nullptr;
+  const e4b_status st = route_scratch_address(&scratch);
+  if (st != E4B_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: the status word and the
+  // last-block counter must start at zero
+  if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return E4B_ERR_CUDA;
+  RouteBuffers b;
+  b.status = reinterpret_cast<int32_t*>(scratch);
+  b.done_counter = reinterpret_cast<uint32_t*>(b.status + 2);
+  b.topk_ids = topk_ids;
+  b.topk_w = topk_w;
+  b.expert_offsets = expert_offsets;
+  b.chunk_off = nullptr;
+  b.block_counts = reinterpret_cast<int32_t*>(scratch + off_counts);
+  b.sorted_slot = sorted_slot;
+  b.slot_pos = reinterpret_cast<int32_t*>(scratch + off_pos);
+  return launch_route(logits, T, E, k, 0, b, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+}

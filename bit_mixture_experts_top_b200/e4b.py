@@ -54,6 +54,7 @@ _SIGS = {
     "e4b_quantize_nf4": ([_vp, _i64, _vp, _vp, _vp], _i32),
     "e4b_route_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "e4b_route": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_route_noalloc": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
     "e4b_moe_workspace_bytes": ([ctypes.POINTER(MoeDesc), _i32], _sz),
     "e4b_moe_workspace_region": ([ctypes.POINTER(MoeDesc), _i32, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz)], _i32),
     "e4b_moe_forward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
@@ -139,6 +140,13 @@ def e4b_route(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_slot, ws
     _check(lib().e4b_route(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
                            _ptr(sorted_slot), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "e4b_route")
+
+
+def e4b_route_noalloc(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_slot, stream=None):
+    """e4b_route with the library's fixed internal scratch instead of a caller workspace."""
+    _need_cuda(logits, topk_ids, topk_w, expert_offsets, sorted_slot)
+    _check(lib().e4b_route_noalloc(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
+                                   _ptr(sorted_slot), _stream(stream)), "e4b_route_noalloc")
 
 
 def e4b_moe_workspace_bytes(desc, T):

@@ -148,6 +148,28 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
                      int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
                      int32_t* sorted_slot, void* ws, size_t ws_bytes, e4b_stream stream);
 
+/*
+ * e4b_route without a caller-provided workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory -- for instance a host runtime that owns all device memory
+ * through its own pool and forbids cudaMalloc once running, or a serving loop
+ * that must not risk an allocation that synchronises the device.
+ *   Arguments and outputs are those of e4b_route, minus ws/ws_bytes.
+ *   Scratch lives in one fixed 1 MiB device array inside the library; every
+ *   GPU that loads the library holds it until the process exits.  Inputs that
+ *   would need more (256 B + 128-token blocks x E x 4 B + T*k x 4 B, e.g. T
+ *   above 16384 at E = 256, k = 8) return E4B_ERR_UNSUPPORTED; nothing runs.
+ *   It allocates nothing: no cudaMalloc, cudaFree or allocating routine.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call on a device shares the one array, so calls that overlap on the
+ *   GPU (different streams, no ordering between them) race and corrupt each
+ *   other's results: order them on one stream or with events.
+ */
+e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
+                             int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                             int32_t* sorted_slot, e4b_stream stream);
+
 /* Workspace bytes e4b_moe_forward needs for this layer at T tokens (0 on a bad desc). */
 size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
 
