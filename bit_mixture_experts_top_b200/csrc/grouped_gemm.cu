@@ -10,10 +10,12 @@
 //   mode 0 (gate_up): G = X_e W_gu[e]^T (+ xa_e B_e), h = silu(G_gate) * G_up -> bf16 [R, I]
 //   mode 1 (down)   : Y = h_e W_dn[e]^T                                       -> fp32 [R, H]
 //
-// B200 design.  The weights are the UMMA M operand (128 rows per tile) and the
-// routed rows of one expert the N operand (tokens_per_tile = BN columns), so a
-// decode batch with a handful of rows per expert still issues full-height
-// MMAs, and one dequantised weight tile serves up to 256 rows in prefill.
+// B200 design.  The weights are the UMMA M operand (128 rows per tile; in
+// tensor memory for decode-sized tiles, in shared memory for prefill tiles)
+// and the routed rows of one expert the N operand (tokens_per_tile = BN
+// columns, in shared memory), so a decode batch with a handful of rows per
+// expert still issues full-height MMAs, and one dequantised weight tile serves
+// up to 256 rows in prefill.
 // One persistent CTA per SM walks a tile list (expert, weight block, row
 // chunk); consecutive tiles share a weight block so its bytes are read from
 // HBM once and from L2 after.  Warp roles:
@@ -23,8 +25,9 @@
 //               B ring;
 //   warp 2      TMEM owner and single-thread UMMA issuer (kind::f16, M=128,
 //               N=BN, K=16, fp32 accumulators in TMEM, two buffers);
-//   warps 3-10  dequant: 4-bit codes + per-block scale -> bf16 written in the
-//               128-byte-swizzled K-major layout the UMMA descriptor reads;
+//   warps 3-10  dequant: 4-bit codes + per-block scale -> bf16 rows written
+//               into tensor memory (tcgen05.st) or 128-byte-swizzled shared
+//               memory, the UMMA A operand;
 //   warps 11-14 epilogue: tcgen05.ld, SwiGLU or fp32 store.
 // Every wait is bounded: on timeout the kernel records E4B_ERR_TIMEOUT, lets
 // copies and MMAs in flight land, frees its TMEM and returns.
@@ -43,7 +46,6 @@ namespace {
 
 constexpr int BM = 128;                      // weight rows per tile (UMMA M)
 constexpr int ATOM_K = 64;                   // K per 128-byte swizzle row of bf16
-constexpr int A_ATOM_BYTES = BM * 128;       // one 128 x 64 bf16 swizzle atom column
 constexpr int RAW_K = 128;                   // K per packed-code stage
 constexpr int RAW_ROW_BYTES = RAW_K / 2;     // 64 bytes of codes per weight row
 constexpr int RAW_STAGE_BYTES = BM * RAW_ROW_BYTES;
@@ -59,19 +61,28 @@ constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
 
-// Decode-sized tiles (BN <= 64) stage 128 K per MMA stage so each dequant
-// thread converts 64 elements per barrier round; prefill tiles (BN >= 128)
-// stage 64 K to leave shared memory for the wide B tiles.
+// Two placements of the dequantised weight tile (the UMMA A operand):
+//  * decode-sized tiles (BN <= 64): A lives in tensor memory.  Columns
+//    [0, 2*BN) hold the two fp32 accumulators, columns [256, 512) a ring of A
+//    stages (64 columns per 128-K stage); shared memory only carries the
+//    packed codes, the activation tiles and the byte LUT.  128 K per stage lets
+//    each dequant thread convert 64 elements per barrier round.
+//  * prefill tiles (BN = 256): A lives in shared memory (128-byte swizzled,
+//    K-major, 64 K per stage), so the two 256-column accumulators can fill
+//    tensor memory and N = 256 MMAs run at the full UMMA rate.
 template <int BN>
 struct Cfg {
-  static constexpr int BKS = BN <= 64 ? 128 : 64;
+  static constexpr bool TMEM_A = BN <= 64;
+  static constexpr int BKS = TMEM_A ? 128 : 64;
   static constexpr int ATOMS = BKS / ATOM_K;
-  static constexpr int A_STAGE_BYTES = ATOMS * A_ATOM_BYTES;
+  static constexpr int A_COLS = BKS / 2;                    // TMEM columns per A stage
+  static constexpr int A_COL0 = 256;                        // first TMEM column of the A ring
+  static constexpr int STAGES = TMEM_A ? (512 - A_COL0) / A_COLS : 3;
+  static constexpr int A_STAGE_BYTES = TMEM_A ? 0 : BM * 128;   // shared-memory A (one atom)
   static constexpr int B_ATOM_BYTES = BN * 128;
   static constexpr int B_STAGE_BYTES = ATOMS * B_ATOM_BYTES;
-  static constexpr int STAGES = BN == 32 ? 2 : (BN == 64 ? 2 : (BN == 128 ? 4 : 3));
-  static constexpr int RAW_STAGES = BN == 32 ? 12 : (BN == 64 ? 10 : (BN == 128 ? 6 : 4));
-  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+  static constexpr int RAW_STAGES = TMEM_A ? 12 : 4;
+  static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_LUT = 0;
   static constexpr int OFF_A = OFF_LUT + LUT_BYTES;
   static constexpr int OFF_B = OFF_A + STAGES * A_STAGE_BYTES;
@@ -81,6 +92,7 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;              // chunk_off and expert_offsets, [E+1] each
   static constexpr int SMEM_BYTES = OFF_TAB + 2 * (kMaxExperts + 1) * 4 + 1024;   // + slack to align the base
+  static_assert(TMEM_A ? 2 * BN <= A_COL0 : 2 * BN <= 512, "accumulators must fit in tensor memory");
   static_assert(B_ATOM_BYTES % 1024 == 0, "B atoms must keep 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -387,15 +399,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&a_full[stage], phase, wctx, 202)) { ok = false; break; }
           if (!mbar_wait(&b_full[stage], phase, wctx, 203)) { ok = false; break; }
           tc_fence_after_sync();
-          const uint32_t a0 = smem_u32(sA + stage * C::A_STAGE_BYTES);
+          const uint32_t a0 = C::TMEM_A ? tmem_base + static_cast<uint32_t>(C::A_COL0 + stage * C::A_COLS)
+                                        : smem_u32(sA + stage * C::A_STAGE_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_STAGE_BYTES);
           // K16 steps: 4 per valid atom; the LoRA step is a single K=16 MMA
           const int nk = ks < mma_steps ? 4 * min(C::ATOMS, (p.K - ks * C::BKS) / ATOM_K) : 1;
           for (int kk = 0; kk < nk; ++kk) {
-            const uint32_t ao = (kk >> 2) * A_ATOM_BYTES + (kk & 3) * 32;
             const uint32_t bo = (kk >> 2) * C::B_ATOM_BYTES + (kk & 3) * 32;
-            umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + ao), smem_desc_sw128(b0 + bo), idesc,
-                         (ks > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (C::TMEM_A)
+              umma_bf16_ts(d_tmem, a0 + kk * 8, smem_desc_sw128(b0 + bo), idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_bf16_ss(d_tmem, smem_desc_sw128(a0 + (kk & 3) * 32), smem_desc_sw128(b0 + bo), idesc,
+                           (ks > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
           issued = true;
@@ -412,9 +427,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp < WARP_EPI0) {
     // ------------------------------------------------------------ dequant
-    const int dt = threadIdx.x - WARP_DQ0 * 32;   // 0..255
-    const int prow = dt & (BM - 1);               // A-tile row written by this thread
-    const int half = dt >> 7;                     // BKS 128: atom; BKS 64: 32-element half of the atom
+    // With A in tensor memory, A row = TMEM lane and a warp may only touch its
+    // own quarter of the lanes; with A in shared memory any mapping works.
+    const int quarter = warp & 3;
+    const int prow = 32 * quarter + lane;          // A-tile row written by this thread
+    const int half = (warp - WARP_DQ0) >> 2;       // BKS 128: atom; BKS 64: 32-element half of the atom
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
     const uint32_t lut_l =
         smem_u32(sLut) + (FMT == E4B_NF4 ? static_cast<uint32_t>(lane & 15) * 8u : static_cast<uint32_t>(lane) * 4u);
     const int kb64 = p.K / 64, kb32 = p.K / 32;
@@ -428,7 +446,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t grow = static_cast<int64_t>(t.e) * p.N + min(wrow, p.N - 1);
       const float* sc_nf4 = reinterpret_cast<const float*>(p.scales) + grow * kb64;
       const uint8_t* sc_mx = reinterpret_cast<const uint8_t*>(p.scales) + grow * kb32;
-      if (C::BKS == 128) {
+      if constexpr (C::BKS == 128) {
         // each thread: 64 elements of its row per stage (atom `half`)
         // scales of this thread's 64 elements: NF4 one absmax, MXFP4 two E8M0 (one per 32)
         auto load_scale = [&](int r, uint64_t& a2, uint32_t& s2a, uint32_t& s2b) {
@@ -451,21 +469,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (r + 1 < raw_steps) load_scale(r + 1, a2n, san, sbn);
           if (!mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
           if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
-          if (r * RAW_K + half * ATOM_K < p.K) {
+          if (r * RAW_K + half * ATOM_K < p.K) {       // warp-uniform (half is per warp)
             const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
-            uint8_t* a = sA + stage * C::A_STAGE_BYTES + half * A_ATOM_BYTES;
+            const uint32_t acol = static_cast<uint32_t>(C::A_COL0 + stage * C::A_COLS + half * 32);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               const uint4 q =
                   *reinterpret_cast<const uint4*>(raw + swizzled_offset(raw_row, half * 2 + c, RAW_ROW_BYTES));
               uint4 o[4];
               dequant32<FMT>(q, lut_l, a2, c == 0 ? sa : sb, o);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4*>(a + swizzled_offset(prow, c * 4 + i, 128)) = o[i];
+              const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
+                                      o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
+              tmem_st_32x32b_x16(t_lane + acol + c * 16, v);
             }
+            tmem_st_wait();
           }
-          fence_proxy_async_smem();
+          tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) {
             mbar_arrive(&a_full[stage]);
@@ -495,10 +514,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               raw + swizzled_offset(raw_row, (ks & 1) * 2 + half, RAW_ROW_BYTES));
           uint4 o[4];
           dequant32<FMT>(q, lut_l, a2, s2, o);
-          uint8_t* a = sA + stage * C::A_STAGE_BYTES;
+          if constexpr (C::TMEM_A) {
+            const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
+                                    o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
+            tmem_st_32x32b_x16(t_lane + static_cast<uint32_t>(C::A_COL0 + stage * C::A_COLS + half * 16), v);
+            tmem_st_wait();
+            tc_fence_before_sync();
+          } else {
+            uint8_t* a = sA + stage * C::A_STAGE_BYTES;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
-          fence_proxy_async_smem();
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
+            fence_proxy_async_smem();
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&a_full[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -511,7 +539,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       if (lora) {                                   // A rows of the LoRA step: B_e[:, wrow]^T, rank padded to 16
         if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 303)) { ok = false; break; }
-        if (half == 0) {
+        if (half == 0) {                              // warp-uniform
           const uint16_t* bcol = p.lora_B + static_cast<int64_t>(t.e) * p.lora_rank * (2 * p.I) + wrow;
           uint32_t v[8];
 #pragma unroll
@@ -520,11 +548,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t hi = (2 * j + 1 < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * j + 1) * 2 * p.I) : 0u;
             v[j] = lo | (hi << 16);
           }
-          uint8_t* a = sA + stage * C::A_STAGE_BYTES;
-          *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 0, 128)) = make_uint4(v[0], v[1], v[2], v[3]);
-          *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 1, 128)) = make_uint4(v[4], v[5], v[6], v[7]);
+          if constexpr (C::TMEM_A) {
+            tmem_st_32x32b_x8(t_lane + static_cast<uint32_t>(C::A_COL0 + stage * C::A_COLS), v);
+            tmem_st_wait();
+          } else {
+            uint8_t* a = sA + stage * C::A_STAGE_BYTES;
+            *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 0, 128)) = make_uint4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 1, 128)) = make_uint4(v[4], v[5], v[6], v[7]);
+          }
         }
-        fence_proxy_async_smem();
+        if constexpr (C::TMEM_A) tc_fence_before_sync();
+        else fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[stage]);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
