@@ -94,7 +94,7 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (d->act != E4B_ACT_SWIGLU) return E4B_ERR_UNSUPPORTED;
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
   const int tpt = d->tokens_per_tile;
-  if (tpt != 0 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 256) return E4B_ERR_UNSUPPORTED;
+  if (tpt != 0 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 192 && tpt != 256) return E4B_ERR_UNSUPPORTED;
   const int64_t R = static_cast<int64_t>(T) * d->k;
   if (R > (int64_t(1) << 30)) return E4B_ERR_UNSUPPORTED;
   // TMA row coordinates are 32-bit: E * 2I rows of codes must fit.
@@ -107,10 +107,12 @@ int32_t pick_tokens_per_tile(const e4b_moe_desc& d, int32_t T) {
   const int64_t R = static_cast<int64_t>(T) * d.k;
   const int64_t active = R < d.E ? R : d.E;
   const int64_t avg = active > 0 ? (R + active - 1) / active : 1;
-  if (avg <= 32) return 32;
-  if (avg <= 64) return 64;
-  if (avg <= 128) return 128;
-  return 256;
+  // smallest tile that holds most experts' rows in one chunk; 192 (not 256)
+  // for prefill keeps the weight tile in tensor memory
+  if (avg <= 16) return 32;
+  if (avg <= 48) return 64;
+  if (avg <= 96) return 128;
+  return 192;
 }
 
 template <typename T>

@@ -62,26 +62,25 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
 
 // Two placements of the dequantised weight tile (the UMMA A operand):
-//  * decode-sized tiles (BN <= 64): A lives in tensor memory.  Columns
-//    [0, 2*BN) hold the two fp32 accumulators, columns [256, 512) a ring of A
-//    stages (64 columns per 128-K stage); shared memory only carries the
-//    packed codes, the activation tiles and the byte LUT.  128 K per stage lets
-//    each dequant thread convert 64 elements per barrier round.
-//  * prefill tiles (BN = 256): A lives in shared memory (128-byte swizzled,
-//    K-major, 64 K per stage), so the two 256-column accumulators can fill
-//    tensor memory and N = 256 MMAs run at the full UMMA rate.
+//  * BN <= 192: A lives in tensor memory.  Columns [0, 2*BN) hold the two
+//    fp32 accumulators, the rest a ring of A stages (BKS/2 columns each);
+//    shared memory only carries the packed codes, the activation tiles and
+//    the byte LUT.  Decode-sized tiles (BN <= 64) stage 128 K so each dequant
+//    thread converts 64 elements per barrier round.
+//  * BN = 256: A lives in shared memory (128-byte swizzled, K-major, 64 K per
+//    stage), so the two 256-column accumulators can fill tensor memory.
 template <int BN>
 struct Cfg {
-  static constexpr bool TMEM_A = BN <= 64;
-  static constexpr int BKS = TMEM_A ? 128 : 64;
+  static constexpr bool TMEM_A = BN != 256;
+  static constexpr int BKS = BN <= 64 ? 128 : 64;
   static constexpr int ATOMS = BKS / ATOM_K;
   static constexpr int A_COLS = BKS / 2;                    // TMEM columns per A stage
-  static constexpr int A_COL0 = 256;                        // first TMEM column of the A ring
+  static constexpr int A_COL0 = 2 * BN > 256 ? 2 * BN : 256;   // first TMEM column of the A ring
   static constexpr int STAGES = TMEM_A ? (512 - A_COL0) / A_COLS : 3;
   static constexpr int A_STAGE_BYTES = TMEM_A ? 0 : BM * 128;   // shared-memory A (one atom)
   static constexpr int B_ATOM_BYTES = BN * 128;
   static constexpr int B_STAGE_BYTES = ATOMS * B_ATOM_BYTES;
-  static constexpr int RAW_STAGES = TMEM_A ? 12 : 4;
+  static constexpr int RAW_STAGES = BN <= 64 ? 12 : (TMEM_A ? 6 : 4);
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_LUT = 0;
   static constexpr int OFF_A = OFF_LUT + LUT_BYTES;
@@ -711,6 +710,7 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
     case 32: return dispatch_fmt_mode<32>(g, tc, ta, tx, prm, s);
     case 64: return dispatch_fmt_mode<64>(g, tc, ta, tx, prm, s);
     case 128: return dispatch_fmt_mode<128>(g, tc, ta, tx, prm, s);
+    case 192: return dispatch_fmt_mode<192>(g, tc, ta, tx, prm, s);
     case 256: return dispatch_fmt_mode<256>(g, tc, ta, tx, prm, s);
     default: return E4B_ERR_UNSUPPORTED;
   }

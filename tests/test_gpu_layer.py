@@ -18,7 +18,7 @@ OSS20 = WORKLOADS["gptoss_20b_mxfp4"]
 OSS120 = WORKLOADS["gptoss_120b_mxfp4_zipf"]
 
 
-@pytest.mark.parametrize("tpt", [0, 32, 64, 128, 256])
+@pytest.mark.parametrize("tpt", [0, 32, 64, 128, 192, 256])
 def test_tiny_mxfp4_layer_every_tile_width(tpt):
     run_and_compare(TINY, 64, tokens_per_tile=tpt)
 
