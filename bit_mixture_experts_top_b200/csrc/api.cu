@@ -94,7 +94,7 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (d->act != E4B_ACT_SWIGLU) return E4B_ERR_UNSUPPORTED;
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
   const int tpt = d->tokens_per_tile;
-  if (tpt != 0 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 192 && tpt != 256) return E4B_ERR_UNSUPPORTED;
+  if (tpt != 0 && tpt != 8 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 192 && tpt != 256) return E4B_ERR_UNSUPPORTED;
   const int64_t R = static_cast<int64_t>(T) * d->k;
   if (R > (int64_t(1) << 30)) return E4B_ERR_UNSUPPORTED;
   // TMA row coordinates are 32-bit: E * 2I rows of codes must fit.
@@ -291,7 +291,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_B = lora_B;
         g.lora_rank = d->lora_rank;
         g.out = h;
-        const e4b_status st = launch_grouped_gemm(g, s);
+        const e4b_status st = tpt == 8 ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
       }
@@ -306,7 +306,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_B = nullptr;
         g.lora_rank = 0;
         g.out = y;
-        const e4b_status st = launch_grouped_gemm(g, s);
+        const e4b_status st = tpt == 8 ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
       }

@@ -67,7 +67,7 @@ struct GroupedGemmLaunch {
   int32_t fmt;              // E4B_NF4 / E4B_MXFP4
   int32_t E, N, K, I;       // stack [E, N, K]; I = intermediate size (mode 0 pairing)
   int32_t R;                // routed rows
-  int32_t tokens_per_tile;  // 32, 64, 128, 256
+  int32_t tokens_per_tile;  // 8 (skinny kernel), 32, 64, 128, 192, 256
   const uint8_t* codes;     // [E, N, K] packed
   const void* scales;
   const uint16_t* act;      // [R, K] bf16 (x_sorted or h)
@@ -81,6 +81,10 @@ struct GroupedGemmLaunch {
   uint64_t wait_limit_ns;
 };
 e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
+
+// Decode-sized batches (tokens_per_tile == 8): warp-level MMA with the codes
+// decoded in registers; chunk_off counts chunks of 8 tokens.
+e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 
 int device_sm_count();
 

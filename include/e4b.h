@@ -83,7 +83,8 @@ typedef struct {
   int32_t lora_rank;       /* 0 = no LoRA; else 1..16 */
   float lora_scale;        /* alpha / r, multiplies the LoRA delta */
   int32_t act;             /* E4B_ACT_SWIGLU */
-  int32_t tokens_per_tile; /* 0 = chosen by the library; else 32, 64, 128, 192 or 256 */
+  int32_t tokens_per_tile; /* 0 = chosen by the library; 8 = decode kernel (warp-level MMA, codes decoded in
+                              registers, chunks of 8 tokens); else 32, 64, 128, 192 or 256 (tcgen05 tiles) */
 } e4b_moe_desc;
 
 /* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */

@@ -18,7 +18,7 @@ OSS20 = WORKLOADS["gptoss_20b_mxfp4"]
 OSS120 = WORKLOADS["gptoss_120b_mxfp4_zipf"]
 
 
-@pytest.mark.parametrize("tpt", [0, 32, 64, 128, 192, 256])
+@pytest.mark.parametrize("tpt", [0, 8, 32, 64, 128, 192, 256])
 def test_tiny_mxfp4_layer_every_tile_width(tpt):
     run_and_compare(TINY, 64, tokens_per_tile=tpt)
 
@@ -36,58 +36,67 @@ def test_tiny_layer_routing_intermediates_bit_exact():
     assert np.array_equal(xs, x[r["sorted_slot"] // TINY.k])
 
 
+@pytest.mark.parametrize("tpt", [0, 8])
 @pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
 @pytest.mark.parametrize("T", [1, 3, 200])
-def test_small_layers_ragged(fmt, T):
-    # several tiles along K and N, a ragged row tail, both formats
+def test_small_layers_ragged(fmt, T, tpt):
+    # several tiles along K and N, a ragged row tail, both formats, both kernels
     w = Workload(f"small_{fmt}", fmt, E=6, H=320, I=192, k=2, tokens=(T,), exp_range=(-4, 2), seed=5)
-    run_and_compare(w, T)
+    run_and_compare(w, T, tokens_per_tile=tpt)
 
 
-def test_k_equals_e_and_one_expert_takes_all():
+@pytest.mark.parametrize("tpt", [0, 8])
+def test_k_equals_e_and_one_expert_takes_all(tpt):
     w = Workload("keqe", "mxfp4", E=8, H=256, I=128, k=8, tokens=(40,), seed=2)
-    run_and_compare(w, 40)
+    run_and_compare(w, 40, tokens_per_tile=tpt)
     w1 = Workload("skew", "nf4", E=16, H=256, I=128, k=2, tokens=(700,), seed=4)
     x, _ = layer.synthetic_tokens(w1, 700)
     lg = np.zeros((700, 16), np.float32)
     lg[:, 3] = 8.0
     lg[:, 9] = 4.0
-    run_and_compare(w1, 700, x=x, logits=synth.to_bf16_bits(lg))   # experts 3 and 9 take every token
+    # experts 3 and 9 take every token
+    run_and_compare(w1, 700, tokens_per_tile=tpt, x=x, logits=synth.to_bf16_bits(lg))
 
 
+@pytest.mark.parametrize("tpt", [0, 8])
 @pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
-def test_lora_tiny_and_zero_b(fmt):
+def test_lora_tiny_and_zero_b(fmt, tpt):
     w = Workload(f"lora_{fmt}", fmt, E=8, H=256, I=128, k=2, tokens=(96,), lora_rank=8, lora_alpha=16.0, seed=6)
-    run_and_compare(w, 96)
+    run_and_compare(w, 96, tokens_per_tile=tpt)
     # B = 0 gives exactly the base layer's output, bit for bit
     dev = device()
-    lay = layer.synthetic_layer(w, dev)
+    lay = layer.synthetic_layer(w, dev, tpt)
     x, logits = layer.synthetic_tokens(w, 96)
     out_l = lay.forward(layer.bits_tensor(x, dev), layer.bits_tensor(logits, dev)).clone()
     lay.lora_B.zero_()
     out_z = lay.forward(layer.bits_tensor(x, dev), layer.bits_tensor(logits, dev)).clone()
-    base = layer.MoeLayer(w.E, w.H, w.I, w.k, fmt, lay.gate_up, lay.down)
+    base = layer.MoeLayer(w.E, w.H, w.I, w.k, fmt, lay.gate_up, lay.down, tokens_per_tile=tpt)
     out_b = base.forward(layer.bits_tensor(x, dev), layer.bits_tensor(logits, dev))
     assert torch.equal(out_z.view(torch.int16), out_b.view(torch.int16))
     assert not torch.equal(out_l.view(torch.int16), out_b.view(torch.int16))
 
 
+@pytest.mark.parametrize("tpt", [0, 8])
 @pytest.mark.parametrize("T", [1, 8])
-def test_qwen3_nf4_decode_full(T):
-    run_and_compare(QWEN, T)
+def test_qwen3_nf4_decode_full(T, tpt):
+    run_and_compare(QWEN, T, tokens_per_tile=tpt)
 
 
-def test_qwen3_nf4_decode_t64_sampled():
-    run_and_compare(QWEN, 64, sample=np.arange(0, 64, 4))
+@pytest.mark.parametrize("tpt", [0, 8, 32])
+def test_qwen3_nf4_decode_t64_sampled(tpt):
+    run_and_compare(QWEN, 64, tokens_per_tile=tpt, sample=np.arange(0, 64, 4))
 
 
-def test_qwen3_lora_t512_sampled():
-    run_and_compare(QWEN_LORA, 512, sample=np.random.default_rng(0).choice(512, 24, replace=False))
+@pytest.mark.parametrize("tpt", [0, 8])
+def test_qwen3_lora_t512_sampled(tpt):
+    run_and_compare(QWEN_LORA, 512, tokens_per_tile=tpt,
+                    sample=np.random.default_rng(0).choice(512, 24, replace=False))
 
 
+@pytest.mark.parametrize("tpt", [0, 8, 32])
 @pytest.mark.parametrize("T", [1, 16])
-def test_gptoss_20b_decode(T):
-    run_and_compare(OSS20, T)
+def test_gptoss_20b_decode(T, tpt):
+    run_and_compare(OSS20, T, tokens_per_tile=tpt)
 
 
 def test_gptoss_20b_prefill_sampled():
