@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "e4b.h"
@@ -85,7 +86,13 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 // Decode-sized batches (tokens_per_tile == 8): warp-level MMA with the codes
 // decoded in registers; chunk_off counts chunks of 8 tokens.
 e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
+bool skinny_gemm_supported(int32_t K, int32_t fmt);   // the per-unit scale buffers fit in shared memory
 
 int device_sm_count();
+
+// 2-D tiled tensor map (inner dim contiguous, `row_bytes` apart) through the
+// driver entry point; false when the driver refuses the description.
+bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
 
 }  // namespace e4b

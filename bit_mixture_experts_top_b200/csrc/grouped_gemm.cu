@@ -616,31 +616,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ---------------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
-               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int BN, int FMT, int MODE>
 e4b_status launch_typed(const GroupedGemmLaunch& g, const CUtensorMap& tc, const CUtensorMap& ta,
                         const CUtensorMap& tx, const Params& prm, cudaStream_t s) {
@@ -672,20 +647,45 @@ e4b_status dispatch_fmt_mode(const GroupedGemmLaunch& g, const CUtensorMap& tc, 
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   if (g.R == 0) return E4B_OK;
   const int BN = g.tokens_per_tile;
   CUtensorMap tc, ta, tx;
   const uint64_t code_rows = static_cast<uint64_t>(g.E) * g.N;
-  if (!encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, RAW_ROW_BYTES,
+  if (!encode_tma_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, RAW_ROW_BYTES,
                  g.mode == 0 ? 64 : BM, CU_TENSOR_MAP_SWIZZLE_64B))
     return E4B_ERR_CUDA;
-  if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, ATOM_K, BN,
+  if (!encode_tma_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, ATOM_K, BN,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return E4B_ERR_CUDA;
   const bool lora = g.mode == 0 && g.lora_rank > 0;
   if (lora) {
-    if (!encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.xa, 64, g.R, 128, ATOM_K, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_tma_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.xa, 64, g.R, 128, ATOM_K, BN, CU_TENSOR_MAP_SWIZZLE_128B))
       return E4B_ERR_CUDA;
   } else {
     tx = ta;

@@ -5,38 +5,51 @@
 // fp32 accumulation, one launch over all experts; "experts4bit-qlora" limits
 // list: the stock epilogue act(gate)*up; "experts4bit-qlora" index table:
 // ExpertsLoRA's per-expert low-rank delta before the activation), organised
-// for the case where each expert sees only a handful of tokens and the weight
-// stream from HBM is the whole cost.
+// for the case where each expert sees only a handful of tokens and streaming
+// the packed weights from HBM is the whole cost.
 //
 // Why a second kernel: with <= 8 tokens per expert a 128-row tcgen05 tile
-// spends one UMMA (fixed issue cost, independent of N) per 1 KB of packed
-// codes, and the dequantised operand must round-trip through shared or tensor
-// memory with a barrier handshake per stage.  Here every warp owns its rows
-// end to end: it streams the packed codes straight into registers, decodes
-// them through a byte table into the A fragments of warp-level bf16 MMAs
-// (m16n8k16, 8 tokens per MMA), and accumulates in registers.  No
-// shared-memory operand, no cross-warp synchronisation.
+// spends one UMMA (a fixed issue cost, whatever N is) per 1 KB of packed codes
+// and hands every dequantised stage from the converting warps to the single
+// MMA thread through a barrier.  Here the decoded weights never leave
+// registers: consumer warps read the packed codes from shared memory, decode
+// them through a byte table straight into the A fragments of warp-level bf16
+// MMAs (m16n8k16, the 8 tokens of a chunk as N) and accumulate in registers.
 //
-// Work unit: (chunk of <= 8 tokens of one expert, group of MT 16-row tiles),
-// full K.  chunk_off[E+1] is the router's prefix of ceil(count_e / 8).
-//  * mode 0 (gate_up): tile j pairs gate rows gi..gi+7 with up rows
-//    I+gi..I+gi+7 (gi = 8 * (MT * rg + j)), so each thread holds gate and up
-//    of the same (token, column) and applies SwiGLU in registers;
-//  * mode 1 (down): tile j covers output rows 16 * (MT * rg + j) + 0..15.
+// Work unit: (chunk of <= 8 tokens of one expert, 128 weight rows), full K.
+// chunk_off[E+1] is the router's prefix of ceil(count_e / 8).
+//  * mode 0 (gate_up): rows are gate columns 64nb..64nb+63 and the matching up
+//    columns I+64nb..; MMA tile t pairs gate rows 8t..8t+7 with up rows
+//    64+8t..64+8t+7, so one thread holds gate and up of the same (token,
+//    column) and applies SwiGLU in registers;
+//  * mode 1 (down): output rows 128nb..128nb+127; tile t = rows 16t..16t+15.
 //
-// Fragment/byte mapping.  Lane (g = lane / 4, c = lane % 4) loads, per 64-K
-// block, the 8 code bytes [8c, 8c+8) of its two rows (g and g+8 of the tile):
-// the four lanes of a quad cover one 32-byte block row, so every load
-// instruction reads whole 32-byte sectors.  MMA i (i = 0..3) of the block
-// takes code byte 2i (elements 16c+4i, +1) as the low K pair and byte 2i+1
-// (elements 16c+4i+2, +3) as the high K pair of the A fragment; the B
-// fragment (activations) is loaded with the same K permutation, so the dot
+// Warp roles (one CTA per SM, persistent):
+//  * warp 8, lane 0, the producer: takes units from a global counter (dynamic,
+//    so every CTA finishes within one unit of the others), warms L2 with the
+//    packed rows of the unit two ahead, copies each unit's scale rows to a
+//    shared buffer (double-buffered per unit; a TMA box with the hardware
+//    swizzle when a scale row is 32, 64 or 128 bytes, else one bulk copy per
+//    contiguous run) and issues the 256-K stages: 128 rows x 128 code bytes
+//    (128-byte swizzle) and the chunk's 8 activation rows x 256 K;
+//  * warps 0-7, consumers: warp (wr, wk) owns MMA tiles 4wr..4wr+3 (64 rows)
+//    and the 64-K block wk of every stage, so the activation fragments it
+//    loads serve 64 rows.  At the end of a unit the four K-partials of each
+//    tile are summed through shared memory and warp (wr, wk) finishes tile
+//    4wr+wk (LoRA step, SwiGLU or the fp32 store).
+//
+// Fragment/byte mapping.  Lane (g = lane / 4, c = lane % 4) takes, per 64-K
+// block, code bytes [8c, 8c+8) of rows g and g+8 of a tile.  MMA i (0..3) of
+// the block uses byte 2i (elements 16c+4i, +1) as the low K pair and byte
+// 2i+1 (elements 16c+4i+2, +3) as the high K pair of the A fragment; the B
+// fragment takes the activations with the same K permutation, so the dot
 // product is unchanged.
 //
-// Scales.  NF4: the byte table holds the bf16-rounded codebook levels; the
-// per-64 fp32 absmax multiplies the block's fp32 partial sum (one MMA chain
-// per block), so the weights are never rounded after scaling.  MXFP4: exact
-// bf16 e2m1 pairs times the bf16 power-of-two scale (exact).
+// Scales.  NF4: the byte table holds the bf16-rounded codebook levels and the
+// fp32 absmax multiplies each block's fp32 partial sum, so the weights are
+// never rounded after scaling.  MXFP4: exact bf16 e2m1 pairs times the bf16
+// power-of-two scale (exact).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -48,48 +61,97 @@
 namespace e4b {
 namespace {
 
-constexpr int SK_WARPS = 8;
-constexpr int SK_THREADS = SK_WARPS * 32;
+constexpr int SK_CONSUMERS = 8;
+constexpr int SK_PRODUCER = 8;                   // warp index
+constexpr int SK_THREADS = 9 * 32;
 constexpr int SK_TOK = 8;                        // tokens per chunk (MMA N)
-constexpr int SK_LUT_WORDS = 256 * 32;           // byte table, one copy per lane
+constexpr int SK_ROWS = 128;                     // weight rows per unit
+constexpr int SK_KST = 256;                      // K per stage
+constexpr int SK_CODE_BYTES = SK_ROWS * SK_KST / 2;          // 16 KB
+constexpr int SK_X_BYTES = SK_TOK * SK_KST * 2;              // 4 KB
+constexpr int SK_STAGE_BYTES = SK_CODE_BYTES + SK_X_BYTES;   // 20 KB
+constexpr int SK_MAX_STAGES = 8;
+constexpr int SK_LUT_BYTES = 256 * 32 * 4;       // byte table, one copy per lane
+constexpr int SK_RED_BYTES = SK_CONSUMERS * 4 * 4 * 32 * 4;  // K-partials of a unit
+constexpr int SK_TAB_BYTES = 2 * (kMaxExperts + 1) * 4;
+constexpr int SK_SMEM_LIMIT = 232448;
 
 struct SkParams {
   int32_t E, N, K, I;
-  int32_t row_groups;     // units per chunk
+  int32_t n_blocks;       // units per chunk
   int32_t lora_rank;
-  const uint8_t* codes;   // [E, N, K/2]
+  int32_t stages;         // ring depth
+  int32_t srow;           // scale bytes per weight row (K/64 fp32 or K/32 e8m0)
+  int32_t scale_bytes;    // bytes of one scale buffer (128 rows, 1024-aligned)
+  int32_t scale_tma;      // 1: scale rows by TMA box (swizzled), 0: bulk copies of the raw runs
+  uint32_t scale_swz;     // XOR mask of the scale buffer's swizzle (0 = none)
+  const uint8_t* codes;   // [E, N, K/2] (L2 warming)
   const void* scales;     // NF4 fp32 [E, N, K/64]; MXFP4 u8 [E, N, K/32]
-  const uint16_t* act;    // [R, K] bf16
   const uint16_t* xa;     // [R, 64] bf16 (mode 0 with LoRA)
   const uint16_t* lora_B; // [E, r, 2I]
   const int32_t* expert_offsets;
   const int32_t* chunk_off;
   void* out;              // mode 0: bf16 h [R, I]; mode 1: fp32 y [R, N]
-  uint32_t lut_hi[8];     // NF4: bf16 levels, two per word (level 2w low, 2w+1 high)
+  int32_t* status;
+  uint32_t* counters;     // [2]: next unit, CTAs done (zero between launches)
+  uint64_t wait_limit_ns;
+  uint32_t level2[8];     // NF4: bf16 levels, two per word (level 2w low half)
 };
 
-__device__ __forceinline__ uint2 ld_stream_v2(const uint8_t* p) {
-  uint2 r;
-  asm("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0, %1}, [%2];"
-               : "=r"(r.x), "=r"(r.y)
-               : "l"(p));
-  return r;
-}
+struct SkLayout {
+  int lut, ring, scale, red, tab, bar, total;
+};
 
-__device__ __forceinline__ uint4 ld_act_v4(const uint16_t* p) {
-  uint4 r;
-  asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
+__host__ __device__ inline SkLayout sk_layout(int stages, int scale_bytes) {
+  SkLayout L;
+  L.lut = 0;
+  L.ring = SK_LUT_BYTES;                                     // 1024-aligned (swizzle atoms)
+  L.scale = L.ring + stages * SK_STAGE_BYTES;
+  L.red = L.scale + 2 * scale_bytes;
+  L.tab = L.red + SK_RED_BYTES;
+  L.bar = L.tab + SK_TAB_BYTES;
+  L.total = L.bar + 256 + 1024;   // barriers, unit ids, NF4 levels; base-alignment slack
+  return L;
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
+// Contiguous global -> shared copy (16-byte aligned, size a multiple of 16),
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // lut_l points at this lane's column of the table (entry stride 32 words).
@@ -113,17 +175,43 @@ __device__ __forceinline__ float e2m1_value(uint32_t nib) {
   return __uint_as_float(((nib & 8u) << 28) | ((nib & 7u) << 22)) * 0x1p126f;
 }
 
+// Warp-uniform bounded wait: every lane polls the barrier (so every lane
+// acquires what the completed phase publishes) and the warp leaves together,
+// either when all lanes saw the phase or when lane 0 found the abort flag or
+// the time limit.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w, int32_t where) {
+  const uint32_t a = smem_u32(bar);
+  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(a, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(a, parity))) return true;
+    if ((it & 15) == 0) {
+      int bad = 0;
+      if ((threadIdx.x & 31) == 0) {
+        if (*w.abort_flag) {
+          bad = 1;
+        } else if (globaltimer_ns() - t0 > w.limit_ns) {
+          *w.abort_flag = 1;
+          record_error(w.status, E4B_ERR_TIMEOUT, where);
+          bad = 1;
+        }
+      }
+      if (__shfl_sync(0xFFFFFFFFu, bad, 0)) return false;
+    }
+  }
+}
+
 struct Unit {
-  int e, t0, m, rg;
+  int e, t0, m, nb;
 };
 
-// Unit u -> (expert, first token, tokens, row group), from the CTA's copies of
-// chunk_off[E+1] and expert_offsets[E+1].
-__device__ __forceinline__ Unit decode_unit(int u, int row_groups, int E, const int32_t* s_chunk,
+// Unit u -> (expert, first token, tokens, weight block), from the CTA's copies
+// of chunk_off[E+1] and expert_offsets[E+1].
+__device__ __forceinline__ Unit decode_unit(int u, int n_blocks, int E, const int32_t* s_chunk,
                                             const int32_t* s_off) {
-  const int chunk = u / row_groups;
+  const int chunk = u / n_blocks;
   Unit r;
-  r.rg = u - chunk * row_groups;
+  r.nb = u - chunk * n_blocks;
   int lo = 0, hi = E;                   // last e with chunk_off[e] <= chunk
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -136,100 +224,11 @@ __device__ __forceinline__ Unit decode_unit(int u, int row_groups, int E, const 
   return r;
 }
 
-template <int FMT, int MODE, int MT>
-struct Slot {
-  uint2 q[MT][2];                                        // code bytes of rows g, g+8 of each tile
-  uint32_t s[MT][2];                                     // NF4 absmax bits / MXFP4 bf16x2 scale
-  uint4 x[2];                                            // 16 activations of token g
-};
-
-// Row of the stack that lane row g of tile 0 reads (tile j, half rr add
-// compile-time multiples of the row steps below).
-template <int MODE, int MT>
-__device__ __forceinline__ int first_row(const SkParams& p, int rg, int g) {
-  return MODE == 0 ? 8 * MT * rg + g : 16 * MT * rg + g;
-}
-
-template <int FMT, int MODE, int MT>
-__device__ __forceinline__ void issue_loads(const SkParams& p, const Unit& u, int b, int g, int c,
-                                            Slot<FMT, MODE, MT>& sl) {
-  const int row0 = first_row<MODE, MT>(p, u.rg, g);
-  const int64_t rbytes = p.K >> 1;
-  const int tile_rows = MODE == 0 ? 8 : 16;             // row step between tiles
-  const int half_rows = MODE == 0 ? p.I : 8;            // row step from row g to row g+8 of a tile
-  const int64_t er = static_cast<int64_t>(u.e) * p.N + row0;
-  const uint8_t* cp = p.codes + er * rbytes + b * 32 + 8 * c;
-#pragma unroll
-  for (int j = 0; j < MT; ++j)
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr)
-      sl.q[j][rr] = ld_stream_v2(cp + (static_cast<int64_t>(j) * tile_rows + rr * half_rows) * rbytes);
-  if (FMT == E4B_NF4) {
-    const int kb = p.K >> 6;
-    const float* sp = static_cast<const float*>(p.scales) + er * kb + b;
-#pragma unroll
-    for (int j = 0; j < MT; ++j)
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-        sl.s[j][rr] = __float_as_uint(__ldg(sp + (static_cast<int64_t>(j) * tile_rows + rr * half_rows) * kb));
-  } else {
-    const int kb = p.K >> 5;
-    const uint8_t* sp = static_cast<const uint8_t*>(p.scales) + er * kb + 2 * b + (c >> 1);
-#pragma unroll
-    for (int j = 0; j < MT; ++j)
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-        sl.s[j][rr] = __ldg(sp + (static_cast<int64_t>(j) * tile_rows + rr * half_rows) * kb);
-  }
-  if (g < u.m) {
-    const uint16_t* xp = p.act + static_cast<int64_t>(u.t0 + g) * p.K + b * 64 + 16 * c;
-    sl.x[0] = ld_act_v4(xp);
-    sl.x[1] = ld_act_v4(xp + 8);
-  } else {
-    sl.x[0] = make_uint4(0, 0, 0, 0);
-    sl.x[1] = make_uint4(0, 0, 0, 0);
-  }
-}
-
-template <int FMT, int MODE, int MT>
-__device__ __forceinline__ void compute_block(const Slot<FMT, MODE, MT>& sl, const uint32_t* lut_l, float (&acc)[MT][4]) {
-  const uint32_t xw[8] = {sl.x[0].x, sl.x[0].y, sl.x[0].z, sl.x[0].w, sl.x[1].x, sl.x[1].y, sl.x[1].z, sl.x[1].w};
-#pragma unroll
-  for (int j = 0; j < MT; ++j) {
-    float blk[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t s2[2] = {0u, 0u};
-    if (FMT == E4B_MXFP4) {
-      s2[0] = e8m0_bf16x2(sl.s[j][0]);
-      s2[1] = e8m0_bf16x2(sl.s[j][1]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t w0 = i < 2 ? sl.q[j][0].x : sl.q[j][0].y;
-      const uint32_t w1 = i < 2 ? sl.q[j][1].x : sl.q[j][1].y;
-      const int by = 2 * (i & 1);
-      uint32_t a[4];
-      a[0] = lut_at(lut_l, w0, by);
-      a[1] = lut_at(lut_l, w1, by);
-      a[2] = lut_at(lut_l, w0, by + 1);
-      a[3] = lut_at(lut_l, w1, by + 1);
-      if (FMT == E4B_MXFP4) {
-        a[0] = bf16x2_mul(a[0], s2[0]);
-        a[1] = bf16x2_mul(a[1], s2[1]);
-        a[2] = bf16x2_mul(a[2], s2[0]);
-        a[3] = bf16x2_mul(a[3], s2[1]);
-        mma_bf16(acc[j], a, xw[2 * i], xw[2 * i + 1]);
-      } else {
-        mma_bf16(blk, a, xw[2 * i], xw[2 * i + 1]);
-      }
-    }
-    if (FMT == E4B_NF4) {
-      const float s0 = __uint_as_float(sl.s[j][0]), s1 = __uint_as_float(sl.s[j][1]);
-      acc[j][0] = fmaf(s0, blk[0], acc[j][0]);
-      acc[j][1] = fmaf(s0, blk[1], acc[j][1]);
-      acc[j][2] = fmaf(s1, blk[2], acc[j][2]);
-      acc[j][3] = fmaf(s1, blk[3], acc[j][3]);
-    }
-  }
+// Stack rows of the two 64-row halves of a unit.
+template <int MODE>
+__device__ __forceinline__ void unit_rows(const SkParams& p, const Unit& u, int& row_a, int& row_b) {
+  row_a = MODE == 0 ? 64 * u.nb : SK_ROWS * u.nb;
+  row_b = MODE == 0 ? p.I + 64 * u.nb : row_a + 64;
 }
 
 __device__ __forceinline__ uint32_t lora_pair(const uint16_t* col, int64_t rstride, int j0, int rank) {
@@ -238,212 +237,390 @@ __device__ __forceinline__ uint32_t lora_pair(const uint16_t* col, int64_t rstri
   return lo | (hi << 16);
 }
 
-template <int MODE, int MT>
-__device__ __forceinline__ void epilogue(const SkParams& p, const Unit& u, int g, int c, float (&acc)[MT][4]) {
-  if (MODE == 0) {
-    if (p.lora_rank > 0) {
-      // LoRA step: A = B_e^T (rows n, K = rank padded to 16), B = xa (scale folded in).
-      uint32_t b0 = 0u, b1 = 0u;
-      if (g < u.m) {
-        const uint32_t* xr = reinterpret_cast<const uint32_t*>(p.xa + static_cast<int64_t>(u.t0 + g) * 64);
-        b0 = __ldg(xr + c);
-        b1 = __ldg(xr + 4 + c);
-      }
-      const int64_t rs = 2 * static_cast<int64_t>(p.I);
-      const uint16_t* Be = p.lora_B + static_cast<int64_t>(u.e) * p.lora_rank * rs;
-#pragma unroll
-      for (int j = 0; j < MT; ++j) {
-        const int col = 8 * (MT * u.rg + j) + g;
-        uint32_t a[4];
-        a[0] = lora_pair(Be + col, rs, 2 * c, p.lora_rank);
-        a[1] = lora_pair(Be + p.I + col, rs, 2 * c, p.lora_rank);
-        a[2] = lora_pair(Be + col, rs, 2 * c + 8, p.lora_rank);
-        a[3] = lora_pair(Be + p.I + col, rs, 2 * c + 8, p.lora_rank);
-        mma_bf16(acc[j], a, b0, b1);
-      }
-    }
-    __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      const int col = 8 * (MT * u.rg + j) + g;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (2 * c + t < u.m) {
-          const float v = acc[j][t], w = acc[j][2 + t];
-          const float sg = __fdividef(v, 1.0f + __expf(-v));
-          h[static_cast<int64_t>(u.t0 + 2 * c + t) * p.I + col] = __float2bfloat16_rn(sg * w);
-        }
-      }
-    }
-  } else {
-    float* y = static_cast<float*>(p.out);
-#pragma unroll
-    for (int j = 0; j < MT; ++j) {
-      const int n = 16 * (MT * u.rg + j) + g;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (2 * c + t < u.m) {
-          float* yr = y + static_cast<int64_t>(u.t0 + 2 * c + t) * p.N + n;
-          yr[0] = acc[j][t];
-          yr[8] = acc[j][2 + t];
-        }
-      }
-    }
-  }
-}
-
-template <int FMT, int MODE, int MT, int D>
-__global__ void __launch_bounds__(SK_THREADS, 2) skinny_gemm_kernel(const __grid_constant__ SkParams p) {
-  extern __shared__ uint32_t sk_smem[];
-  uint32_t* lut = sk_smem;
-  int32_t* s_chunk = reinterpret_cast<int32_t*>(sk_smem + SK_LUT_WORDS);
+template <int FMT, int MODE>
+__global__ void __launch_bounds__(SK_THREADS, 1)
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                       const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ SkParams p) {
+  extern __shared__ uint8_t sk_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sk_dyn) + 1023) & ~uintptr_t(1023));
+  const SkLayout L = sk_layout(p.stages, p.scale_bytes);
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
+  uint8_t* ring = smem + L.ring;
+  uint8_t* sbuf = smem + L.scale;
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  int32_t* s_chunk = reinterpret_cast<int32_t*>(smem + L.tab);
   int32_t* s_off = s_chunk + (kMaxExperts + 1);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
+  uint64_t* empty = full + SK_MAX_STAGES;
+  uint64_t* sfull = empty + SK_MAX_STAGES;      // [2]
+  uint64_t* sempty = sfull + 2;                 // [2]
+  uint64_t* rfull = sempty + 2;
+  uint64_t* rempty = rfull + 1;
+  int32_t* s_unit = reinterpret_cast<int32_t*>(rempty + 1);   // [2]
+  int32_t* s_abort = s_unit + 2;
+  uint16_t* s_level = reinterpret_cast<uint16_t*>(smem + L.bar + 192);   // [16]
 
-  __shared__ uint16_t s_level[16];
-  if (FMT == E4B_NF4 && threadIdx.x < 16) {
-    const uint32_t w = p.lut_hi[threadIdx.x >> 1];
-    s_level[threadIdx.x] = static_cast<uint16_t>(w >> (16 * (threadIdx.x & 1)));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], SK_CONSUMERS);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sfull[b], 1);
+      mbar_init(&sempty[b], SK_CONSUMERS);
+    }
+    mbar_init(rfull, SK_CONSUMERS);
+    mbar_init(rempty, SK_CONSUMERS);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (FMT == E4B_NF4 && threadIdx.x < 16)
+    s_level[threadIdx.x] = static_cast<uint16_t>(p.level2[threadIdx.x >> 1] >> (16 * (threadIdx.x & 1)));
+  for (int i = threadIdx.x; i <= p.E; i += SK_THREADS) {
+    s_chunk[i] = __ldg(p.chunk_off + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
+  }
+  if (warp == SK_PRODUCER && lane == 0) {
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_x);
+    if (p.scale_tma) tma_prefetch_desc(&tm_scales);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < SK_LUT_WORDS; i += SK_THREADS) {
+  // Byte -> bf16 pair table, one copy per lane so every lane reads its own bank.
+  for (int i = threadIdx.x; i < 256 * 32; i += SK_THREADS) {
     const uint32_t b = static_cast<uint32_t>(i) >> 5;
     uint32_t v;
-    if (FMT == E4B_NF4) {
-      // element 2j sits in the high nibble: it goes to the low half
+    if (FMT == E4B_NF4) {   // element 2j in the high nibble -> low half
       v = static_cast<uint32_t>(s_level[b >> 4]) | (static_cast<uint32_t>(s_level[b & 15u]) << 16);
-    } else {
-      // element 2j sits in the low nibble: it goes to the low half
+    } else {                // element 2j in the low nibble -> low half
       __nv_bfloat162 t = __floats2bfloat162_rn(e2m1_value(b & 15u), e2m1_value(b >> 4));
       v = *reinterpret_cast<uint32_t*>(&t);
     }
     lut[i] = v;
   }
-  for (int i = threadIdx.x; i <= p.E; i += SK_THREADS) {
-    s_chunk[i] = __ldg(p.chunk_off + i);
-    s_off[i] = __ldg(p.expert_offsets + i);
-  }
   __syncthreads();
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const uint32_t* lut_l = lut + lane;
-  const int gwarp = blockIdx.x * SK_WARPS + warp;
-  const int nwarps = gridDim.x * SK_WARPS;
-  const int total = s_chunk[p.E] * p.row_groups;
-  if (gwarp >= total) return;
+  const WaitCtx wctx{s_abort, p.status, p.wait_limit_ns};
+  const int total = s_chunk[p.E] * p.n_blocks;
   const int KB = p.K >> 6;
-  const int my_units = (total - gwarp + nwarps - 1) / nwarps;
-  const int nsteps = my_units * KB;
+  const int nst = (p.K + SK_KST - 1) / SK_KST;
 
-  // load side: next step to issue, its unit and block
-  int l_unit = gwarp, l_b = 0;
-  Unit lu = decode_unit(l_unit, p.row_groups, p.E, s_chunk, s_off);
-  // compute side
-  int c_unit = gwarp, c_b = 0;
-  Unit cu = lu;
-
-  Slot<FMT, MODE, MT> slot[D];
-  float acc[MT][4];
-#pragma unroll
-  for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-
-  auto advance_load = [&]() {
-    if (++l_b == KB) {
-      l_b = 0;
-      l_unit += nwarps;
-      if (l_unit < total) lu = decode_unit(l_unit, p.row_groups, p.E, s_chunk, s_off);
-    }
-  };
-
-#pragma unroll
-  for (int d = 0; d < D; ++d) {
-    if (d < nsteps) {
-      issue_loads<FMT, MODE, MT>(p, lu, l_b, g, c, slot[d]);
-      advance_load();
-    }
-  }
-
-  for (int s0 = 0; s0 < nsteps; s0 += D) {
-#pragma unroll
-    for (int d = 0; d < D; ++d) {
-      const int st = s0 + d;
-      if (st < nsteps) {
-        compute_block<FMT, MODE, MT>(slot[d], lut_l, acc);
-        if (st + D < nsteps) {
-          issue_loads<FMT, MODE, MT>(p, lu, l_b, g, c, slot[d]);
-          advance_load();
+  if (warp == SK_PRODUCER) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool drained = false;
+      auto fetch = [&]() {
+        if (drained) return total;
+        const int u = static_cast<int>(atomicAdd(&p.counters[0], 1u));
+        if (u >= total) drained = true;
+        return u < total ? u : total;
+      };
+      // packed rows of a unit: two contiguous runs; warm L2 with them two units ahead
+      auto warm = [&](int u) {
+        if (u >= total) return;
+        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+        int row_a, row_b;
+        unit_rows<MODE>(p, un, row_a, row_b);
+        for (int half = 0; half < 2; ++half) {
+          const int row0 = half == 0 ? row_a : row_b;
+          const int nrows = min(64, p.N - row0);
+          if (nrows > 0)
+            bulk_prefetch_l2(p.codes + (static_cast<int64_t>(un.e) * p.N + row0) * (p.K / 2),
+                             static_cast<uint32_t>(nrows) * (p.K / 2));
         }
-        if (++c_b == KB) {
-          epilogue<MODE, MT>(p, cu, g, c, acc);
+      };
+      int q0 = fetch(), q1 = fetch();
+      warm(q0);
+      warm(q1);
+      int sb = 0, slot = 0;
+      uint32_t sph = 0, ph = 0, armed = 0, par = 0, sarmed = 0, spar = 0;
+      bool ok = true;
+      for (;;) {
+        const int u = q0;
+        q0 = q1;
+        q1 = fetch();
+        warm(q1);
+        if (!mbar_wait(&sempty[sb], sph ^ 1u, wctx, 711)) { ok = false; break; }
+        if (u >= total) {
+          s_unit[sb] = -1;
+          mbar_arrive(&sfull[sb]);
+          break;
+        }
+        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+        int row_a, row_b;
+        unit_rows<MODE>(p, un, row_a, row_b);
+        const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
+        // the unit's scale rows (64 + 64), each half one contiguous 16-byte aligned run
+        s_unit[sb] = u;
+        uint8_t* sdst = sbuf + sb * p.scale_bytes;
+        if (p.scale_tma) {
+          mbar_arrive_expect_tx(&sfull[sb], 2 * 64 * p.srow);
+          tma_load_2d(sdst, &tm_scales, &sfull[sb], 0, ya);
+          tma_load_2d(sdst + 64 * p.srow, &tm_scales, &sfull[sb], 0, yb);
+        } else {
+          const int na = max(0, min(64, p.N - row_a)), nb = max(0, min(64, p.N - row_b));
+          mbar_arrive_expect_tx(&sfull[sb], (na + nb) * p.srow);
+          const uint8_t* sc = static_cast<const uint8_t*>(p.scales);
+          if (na) bulk_copy_g2s(sdst, sc + static_cast<int64_t>(ya) * p.srow, na * p.srow, &sfull[sb]);
+          if (nb) bulk_copy_g2s(sdst + 64 * p.srow, sc + static_cast<int64_t>(yb) * p.srow, nb * p.srow, &sfull[sb]);
+        }
+        sarmed |= 1u << sb;
+        spar = (spar & ~(1u << sb)) | (sph << sb);
+        for (int st = 0; st < nst; ++st) {
+          if (!mbar_wait(&empty[slot], ph ^ 1u, wctx, 712)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[slot], SK_STAGE_BYTES);
+          uint8_t* dst = ring + slot * SK_STAGE_BYTES;
+          tma_load_2d(dst, &tm_codes, &full[slot], SK_KST / 2 * st, ya);
+          tma_load_2d(dst + SK_CODE_BYTES / 2, &tm_codes, &full[slot], SK_KST / 2 * st, yb);
 #pragma unroll
-          for (int j = 0; j < MT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-          c_b = 0;
-          c_unit += nwarps;
-          if (c_unit < total) cu = decode_unit(c_unit, p.row_groups, p.E, s_chunk, s_off);
+          for (int i = 0; i < 4; ++i)
+            tma_load_2d(dst + SK_CODE_BYTES + 1024 * i, &tm_x, &full[slot], SK_KST * st + 64 * i, un.t0);
+          armed |= 1u << slot;
+          par = (par & ~(1u << slot)) | (ph << slot);
+          if (++slot == p.stages) { slot = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        if (++sb == 2) { sb = 0; sph ^= 1u; }
+      }
+      while (!drained) (void)fetch();
+      // the last CTA through resets the counters for the next launch
+      __threadfence();
+      if (atomicAdd(&p.counters[1], 1u) == gridDim.x - 1) {
+        atomicExch(&p.counters[0], 0u);
+        atomicExch(&p.counters[1], 0u);
+      }
+      if (!ok) {   // let every issued copy land before the CTA's shared memory is released
+        for (int s = 0; s < p.stages; ++s)
+          if (armed & (1u << s)) mbar_drain(&full[s], (par >> s) & 1u, p.wait_limit_ns);
+        for (int b = 0; b < 2; ++b)
+          if (sarmed & (1u << b)) mbar_drain(&sfull[b], (spar >> b) & 1u, p.wait_limit_ns);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int wr = warp >> 2, wk = warp & 3;
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t* lut_l = lut + lane;
+    const uint32_t ring_s = smem_u32(ring);
+    int sb = 0, slot = 0;
+    uint32_t sph = 0, ph = 0, rph = 0;
+    bool ok = true;
+    for (;;) {
+      if (!warp_wait(&sfull[sb], sph, wctx, 721)) break;
+      const int u = s_unit[sb];
+      if (u < 0) break;
+      const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+      const uint32_t sc_s = smem_u32(sbuf + sb * p.scale_bytes);
+      float acc[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int st = 0; st < nst; ++st) {
+        if (!warp_wait(&full[slot], ph, wctx, 722)) { ok = false; break; }
+        const int blk = 4 * st + wk;
+        if (blk < KB) {
+          const uint32_t cs = ring_s + slot * SK_STAGE_BYTES;
+          const uint32_t xs = cs + SK_CODE_BYTES + 1024 * wk + 128 * g;
+          const uint4 xa = lds128(xs + 16 * ((2 * c) ^ g));
+          const uint4 xb = lds128(xs + 16 * ((2 * c + 1) ^ g));
+          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          const uint32_t half8 = 8 * (c & 1);
+          const uint32_t chunk = 2 * wk + (c >> 1);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = 4 * wr + j;
+            const int r0 = MODE == 0 ? 8 * t + g : 16 * t + g;
+            const int r1 = MODE == 0 ? 64 + 8 * t + g : 16 * t + 8 + g;
+            const uint2 q0 = lds64(cs + 128 * r0 + 16 * (chunk ^ g) + half8);
+            const uint2 q1 = lds64(cs + 128 * r1 + 16 * (chunk ^ g) + half8);
+            uint32_t o0 = r0 * p.srow + blk * (FMT == E4B_NF4 ? 4 : 2);
+            uint32_t o1 = r1 * p.srow + blk * (FMT == E4B_NF4 ? 4 : 2);
+            o0 ^= (o0 >> 3) & p.scale_swz;
+            o1 ^= (o1 >> 3) & p.scale_swz;
+            const uint32_t s0 = FMT == E4B_NF4 ? lds32(sc_s + o0) : lds16(sc_s + o0);
+            const uint32_t s1 = FMT == E4B_NF4 ? lds32(sc_s + o1) : lds16(sc_s + o1);
+            if (FMT == E4B_NF4) {
+              float bs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t w0 = i < 2 ? q0.x : q0.y, w1 = i < 2 ? q1.x : q1.y;
+                const int by = 2 * (i & 1);
+                const uint32_t a[4] = {lut_at(lut_l, w0, by), lut_at(lut_l, w1, by), lut_at(lut_l, w0, by + 1),
+                                       lut_at(lut_l, w1, by + 1)};
+                mma_bf16(bs, a, xw[2 * i], xw[2 * i + 1]);
+              }
+              const float f0 = __uint_as_float(s0), f1 = __uint_as_float(s1);
+              acc[j][0] = fmaf(f0, bs[0], acc[j][0]);
+              acc[j][1] = fmaf(f0, bs[1], acc[j][1]);
+              acc[j][2] = fmaf(f1, bs[2], acc[j][2]);
+              acc[j][3] = fmaf(f1, bs[3], acc[j][3]);
+            } else {
+              const uint32_t e0 = e8m0_bf16x2((s0 >> (8 * (c >> 1))) & 0xFFu);
+              const uint32_t e1 = e8m0_bf16x2((s1 >> (8 * (c >> 1))) & 0xFFu);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t w0 = i < 2 ? q0.x : q0.y, w1 = i < 2 ? q1.x : q1.y;
+                const int by = 2 * (i & 1);
+                const uint32_t a[4] = {bf16x2_mul(lut_at(lut_l, w0, by), e0), bf16x2_mul(lut_at(lut_l, w1, by), e1),
+                                       bf16x2_mul(lut_at(lut_l, w0, by + 1), e0),
+                                       bf16x2_mul(lut_at(lut_l, w1, by + 1), e1)};
+                mma_bf16(acc[j], a, xw[2 * i], xw[2 * i + 1]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (++slot == p.stages) { slot = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[sb]);
+      // sum the four K-partials of each tile; warp (wr, wk) finishes tile 4wr+wk
+      if (!warp_wait(rempty, rph ^ 1u, wctx, 723)) break;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red[((warp * 4 + j) * 4 + i) * 32 + lane] = acc[j][i];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rfull);
+      if (!warp_wait(rfull, rph, wctx, 724)) break;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] += red[(((4 * wr + k) * 4 + wk) * 4 + i) * 32 + lane];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rempty);
+      rph ^= 1u;
+      const int t = 4 * wr + wk;
+      if (MODE == 0) {
+        const int col = 64 * un.nb + 8 * t + g;
+        if (p.lora_rank > 0) {
+          // LoRA step: A = B_e^T (rows n, K = rank padded to 16), B = xa (scale folded in)
+          uint32_t b0 = 0u, b1 = 0u;
+          if (g < un.m) {
+            const uint32_t* xr = reinterpret_cast<const uint32_t*>(p.xa + static_cast<int64_t>(un.t0 + g) * 64);
+            b0 = __ldg(xr + c);
+            b1 = __ldg(xr + 4 + c);
+          }
+          const int64_t rs = 2 * static_cast<int64_t>(p.I);
+          const uint16_t* Be = p.lora_B + static_cast<int64_t>(un.e) * p.lora_rank * rs;
+          const uint32_t a[4] = {lora_pair(Be + col, rs, 2 * c, p.lora_rank),
+                                 lora_pair(Be + p.I + col, rs, 2 * c, p.lora_rank),
+                                 lora_pair(Be + col, rs, 2 * c + 8, p.lora_rank),
+                                 lora_pair(Be + p.I + col, rs, 2 * c + 8, p.lora_rank)};
+          mma_bf16(v, a, b0, b1);
+        }
+        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (2 * c + q < un.m) {
+            const float gt = v[q], up = v[2 + q];
+            const float sg = __fdividef(gt, 1.0f + __expf(-gt));
+            h[static_cast<int64_t>(un.t0 + 2 * c + q) * p.I + col] = __float2bfloat16_rn(sg * up);
+          }
+        }
+      } else {
+        const int n = SK_ROWS * un.nb + 16 * t + g;
+        float* y = static_cast<float*>(p.out);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          if (2 * c + q < un.m) {
+            float* yr = y + static_cast<int64_t>(un.t0 + 2 * c + q) * p.N + n;
+            if (n < p.N) yr[0] = v[q];
+            if (n + 8 < p.N) yr[8] = v[2 + q];
+          }
         }
       }
+      if (++sb == 2) { sb = 0; sph ^= 1u; }
     }
   }
 }
 
-constexpr int kSmemBytes = SK_LUT_WORDS * 4 + 2 * (kMaxExperts + 1) * 4;
-
-template <int FMT, int MODE, int MT, int D>
-e4b_status launch_cfg(const SkParams& prm, cudaStream_t s) {
-  auto kern = skinny_gemm_kernel<FMT, MODE, MT, D>;
-  static int blocks_per_sm[64] = {0};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return E4B_ERR_CUDA;
-  int bps = 0;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (blocks_per_sm[dev] == 0) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
-        return E4B_ERR_CUDA;
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, SK_THREADS, kSmemBytes) != cudaSuccess || n < 1)
-        return E4B_ERR_CUDA;
-      blocks_per_sm[dev] = n;
-    }
-    bps = blocks_per_sm[dev];
-  }
-  kern<<<device_sm_count() * bps, SK_THREADS, kSmemBytes, s>>>(prm);
+template <int FMT, int MODE>
+e4b_status launch_typed(const CUtensorMap& tc, const CUtensorMap& tx, const CUtensorMap& ts, const SkParams& prm,
+                        int smem, cudaStream_t s) {
+  auto kern = skinny_gemm_kernel<FMT, MODE>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_SMEM_LIMIT);
+  });
+  if (attr_err != cudaSuccess) return E4B_ERR_CUDA;
+  kern<<<device_sm_count(), SK_THREADS, smem, s>>>(tc, tx, ts, prm);
   return cudaGetLastError() == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }
 
+int scale_row_bytes(int32_t K, int32_t fmt) { return fmt == E4B_NF4 ? K / 16 : K / 32; }
+int scale_buffer_bytes(int32_t K, int32_t fmt) { return (SK_ROWS * scale_row_bytes(K, fmt) + 1023) & ~1023; }
+
 }  // namespace
+
+bool skinny_gemm_supported(int32_t K, int32_t fmt) {
+  return sk_layout(3, scale_buffer_bytes(K, fmt)).total <= SK_SMEM_LIMIT;
+}
 
 e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   if (g.R == 0) return E4B_OK;
-  constexpr int MT = 2;
+  if (g.K % 64 != 0 || (g.mode == 0 && g.I % 64 != 0) || !skinny_gemm_supported(g.K, g.fmt))
+    return E4B_ERR_UNSUPPORTED;
   SkParams prm;
   prm.E = g.E;
   prm.N = g.N;
   prm.K = g.K;
   prm.I = g.I;
-  prm.row_groups = g.mode == 0 ? g.I / (8 * MT) : g.N / (16 * MT);
+  prm.n_blocks = g.mode == 0 ? g.I / 64 : (g.N + SK_ROWS - 1) / SK_ROWS;
   prm.lora_rank = g.mode == 0 ? g.lora_rank : 0;
+  prm.srow = scale_row_bytes(g.K, g.fmt);
+  prm.scale_bytes = scale_buffer_bytes(g.K, g.fmt);
+  // scale rows of 32, 64 or 128 bytes go through a swizzled TMA box, so the
+  // eight rows a fragment reads fall in different banks
+  prm.scale_tma = (prm.srow == 32 || prm.srow == 64 || prm.srow == 128) ? 1 : 0;
+  prm.scale_swz = prm.scale_tma ? static_cast<uint32_t>(((prm.srow >> 4) - 1) << 4) : 0u;
+  int stages = SK_MAX_STAGES;
+  while (stages > 3 && sk_layout(stages, prm.scale_bytes).total > SK_SMEM_LIMIT) --stages;
+  prm.stages = stages;
   prm.codes = g.codes;
   prm.scales = g.scales;
-  prm.act = g.act;
   prm.xa = g.xa;
   prm.lora_B = g.lora_B;
   prm.expert_offsets = g.expert_offsets;
   prm.chunk_off = g.chunk_off;
   prm.out = g.out;
+  prm.status = g.status;
+  prm.counters = reinterpret_cast<uint32_t*>(g.status) + 8 + 2 * g.mode;
+  prm.wait_limit_ns = g.wait_limit_ns;
   const Nf4Table& t = nf4_table();
   for (int w = 0; w < 8; ++w) {
     const __nv_bfloat16 lo = __float2bfloat16_rn(t.level[2 * w]);
     const __nv_bfloat16 hi = __float2bfloat16_rn(t.level[2 * w + 1]);
-    prm.lut_hi[w] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&lo)) |
+    prm.level2[w] = static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&lo)) |
                     (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(&hi)) << 16);
   }
-  if ((g.mode == 0 && g.I % (8 * MT) != 0) || (g.mode == 1 && g.N % (16 * MT) != 0) || g.K % 64 != 0)
-    return E4B_ERR_UNSUPPORTED;
+  CUtensorMap tc, tx, ts;
+  const uint64_t code_rows = static_cast<uint64_t>(g.E) * g.N;
+  if (!encode_tma_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, SK_KST / 2, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return E4B_ERR_CUDA;
+  if (!encode_tma_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, 64,
+                     SK_TOK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return E4B_ERR_CUDA;
+  if (prm.scale_tma) {
+    const CUtensorMapSwizzle sw = prm.srow == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : prm.srow == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                   : CU_TENSOR_MAP_SWIZZLE_32B;
+    if (!encode_tma_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.scales, prm.srow, code_rows, prm.srow, prm.srow, 64, sw))
+      return E4B_ERR_CUDA;
+  } else {
+    ts = tc;
+  }
+  const int smem = sk_layout(stages, prm.scale_bytes).total;
   if (g.fmt == E4B_NF4)
-    return g.mode == 0 ? launch_cfg<E4B_NF4, 0, MT, 4>(prm, s) : launch_cfg<E4B_NF4, 1, MT, 4>(prm, s);
-  return g.mode == 0 ? launch_cfg<E4B_MXFP4, 0, MT, 4>(prm, s) : launch_cfg<E4B_MXFP4, 1, MT, 4>(prm, s);
+    return g.mode == 0 ? launch_typed<E4B_NF4, 0>(tc, tx, ts, prm, smem, s)
+                       : launch_typed<E4B_NF4, 1>(tc, tx, ts, prm, smem, s);
+  return g.mode == 0 ? launch_typed<E4B_MXFP4, 0>(tc, tx, ts, prm, smem, s)
+                     : launch_typed<E4B_MXFP4, 1>(tc, tx, ts, prm, smem, s);
 }
 
 }  // namespace e4b
