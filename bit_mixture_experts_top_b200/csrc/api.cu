@@ -94,6 +94,8 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (d->act != E4B_ACT_SWIGLU) return E4B_ERR_UNSUPPORTED;
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
   const int tpt = d->tokens_per_tile;
+  if (tpt == 8 && !(skinny_gemm_supported(d->H, d->format) && skinny_gemm_supported(d->I, d->format)))
+    return E4B_ERR_UNSUPPORTED;
   if (tpt != 0 && tpt != 8 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 192 && tpt != 256) return E4B_ERR_UNSUPPORTED;
   const int64_t R = static_cast<int64_t>(T) * d->k;
   if (R > (int64_t(1) << 30)) return E4B_ERR_UNSUPPORTED;
@@ -107,8 +109,10 @@ int32_t pick_tokens_per_tile(const e4b_moe_desc& d, int32_t T) {
   const int64_t R = static_cast<int64_t>(T) * d.k;
   const int64_t active = R < d.E ? R : d.E;
   const int64_t avg = active > 0 ? (R + active - 1) / active : 1;
-  // smallest tile that holds most experts' rows in one chunk; 192 (not 256)
-  // for prefill keeps the weight tile in tensor memory
+  // a handful of rows per expert: the decode kernel (weight stream bound);
+  // else the smallest tcgen05 tile that holds most experts' rows in one chunk,
+  // 192 (not 256) for prefill keeps the weight tile in tensor memory
+  if (avg <= 12 && skinny_gemm_supported(d.H, d.format) && skinny_gemm_supported(d.I, d.format)) return 8;
   if (avg <= 16) return 32;
   if (avg <= 48) return 64;
   if (avg <= 96) return 128;

@@ -25,21 +25,21 @@
 //  * mode 1 (down): output rows 128nb..128nb+127; tile t = rows 16t..16t+15.
 //
 // Warp roles (one CTA per SM, persistent):
-//  * warp 8, lane 0, the producer: takes units from a global counter (dynamic,
-//    so every CTA finishes within one unit of the others), warms L2 with the
-//    packed rows of the unit two ahead, copies each unit's scale rows to a
-//    shared buffer (double-buffered per unit; a TMA box with the hardware
+//  * warp 16, lane 0, the producer: takes units from a global counter (dynamic,
+//    so every CTA finishes within one unit of the others), copies each unit's
+//    scale rows to a shared buffer one unit ahead (2 buffers; a TMA box with the hardware
 //    swizzle when a scale row is 32, 64 or 128 bytes, else one bulk copy per
 //    contiguous run) and issues the 256-K stages: 128 rows x 128 code bytes
 //    (128-byte swizzle) and the chunk's 8 activation rows x 256 K;
-//  * warps 0-7, consumers: warp (wr, wk) owns MMA tiles 4wr..4wr+3 (64 rows)
+//  * warps 0-15, consumers: warp (wr, wk) owns MMA tiles 2wr, 2wr+1 (32 rows)
 //    and the 64-K block wk of every stage, so the activation fragments it
-//    loads serve 64 rows.  At the end of a unit the four K-partials of each
-//    tile are summed through shared memory and warp (wr, wk) finishes tile
-//    4wr+wk (LoRA step, SwiGLU or the fp32 store).
+//    loads serve 32 rows.  At the end of a unit the four K-partials of each
+//    tile are summed through shared memory and warp (wr, wk < 2) finishes
+//    tile 2wr+wk (LoRA step, SwiGLU or the fp32 store).
 //
 // Fragment/byte mapping.  Lane (g = lane / 4, c = lane % 4) takes, per 64-K
-// block, code bytes [8c, 8c+8) of rows g and g+8 of a tile.  MMA i (0..3) of
+// block, code bytes [8c, 8c+8) of fragment rows g and g+8 of a tile (fragment
+// row g is tile row rho(g) = 2(g mod 4) + g/4, a bank-spreading permutation).  MMA i (0..3) of
 // the block uses byte 2i (elements 16c+4i, +1) as the low K pair and byte
 // 2i+1 (elements 16c+4i+2, +3) as the high K pair of the A fragment; the B
 // fragment takes the activations with the same K permutation, so the dot
@@ -61,9 +61,11 @@
 namespace e4b {
 namespace {
 
-constexpr int SK_CONSUMERS = 8;
-constexpr int SK_PRODUCER = 8;                   // warp index
-constexpr int SK_THREADS = 9 * 32;
+constexpr int SK_CONSUMERS = 16;
+constexpr int SK_PRODUCER = 16;                  // warp index
+constexpr int SK_THREADS = 17 * 32;
+constexpr int SK_TPW = 2;                        // MMA tiles per consumer warp
+constexpr int SK_SBUF = 2;                       // per-unit scale buffers
 constexpr int SK_TOK = 8;                        // tokens per chunk (MMA N)
 constexpr int SK_ROWS = 128;                     // weight rows per unit
 constexpr int SK_KST = 256;                      // K per stage
@@ -71,8 +73,11 @@ constexpr int SK_CODE_BYTES = SK_ROWS * SK_KST / 2;          // 16 KB
 constexpr int SK_X_BYTES = SK_TOK * SK_KST * 2;              // 4 KB
 constexpr int SK_STAGE_BYTES = SK_CODE_BYTES + SK_X_BYTES;   // 20 KB
 constexpr int SK_MAX_STAGES = 8;
-constexpr int SK_LUT_BYTES = 256 * 32 * 4;       // byte table, one copy per lane
-constexpr int SK_RED_BYTES = SK_CONSUMERS * 4 * 4 * 32 * 4;  // K-partials of a unit
+// byte table: entry b holds one copy per lane at 256*b + 4*lane (the upper
+// 128 bytes of each entry are unused), so a single byte permute of the code
+// word and the lane offset forms the address
+constexpr int SK_LUT_BYTES = 256 * 256;
+constexpr int SK_RED_BYTES = SK_CONSUMERS * SK_TPW * 4 * 32 * 4;  // K-partials of a unit
 constexpr int SK_TAB_BYTES = 2 * (kMaxExperts + 1) * 4;
 constexpr int SK_SMEM_LIMIT = 232448;
 
@@ -85,7 +90,7 @@ struct SkParams {
   int32_t scale_bytes;    // bytes of one scale buffer (128 rows, 1024-aligned)
   int32_t scale_tma;      // 1: scale rows by TMA box (swizzled), 0: bulk copies of the raw runs
   uint32_t scale_swz;     // XOR mask of the scale buffer's swizzle (0 = none)
-  const uint8_t* codes;   // [E, N, K/2] (L2 warming)
+  const uint8_t* codes;   // [E, N, K/2]
   const void* scales;     // NF4 fp32 [E, N, K/64]; MXFP4 u8 [E, N, K/32]
   const uint16_t* xa;     // [R, 64] bf16 (mode 0 with LoRA)
   const uint16_t* lora_B; // [E, r, 2I]
@@ -107,11 +112,19 @@ __host__ __device__ inline SkLayout sk_layout(int stages, int scale_bytes) {
   L.lut = 0;
   L.ring = SK_LUT_BYTES;                                     // 1024-aligned (swizzle atoms)
   L.scale = L.ring + stages * SK_STAGE_BYTES;
-  L.red = L.scale + 2 * scale_bytes;
+  L.red = L.scale + SK_SBUF * scale_bytes;
   L.tab = L.red + SK_RED_BYTES;
   L.bar = L.tab + SK_TAB_BYTES;
   L.total = L.bar + 256 + 1024;   // barriers, unit ids, NF4 levels; base-alignment slack
   return L;
+}
+
+// d = A * B (accumulator starts at zero)
+__device__ __forceinline__ void mma_bf16_z(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -119,30 +132,6 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
-  return v;
 }
 
 // Contiguous global -> shared copy (16-byte aligned, size a multiple of 16),
@@ -154,9 +143,10 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
                : "memory");
 }
 
-// lut_l points at this lane's column of the table (entry stride 32 words).
-__device__ __forceinline__ uint32_t lut_at(const uint32_t* lut_l, uint32_t word, int byte) {
-  return lut_l[((word >> (8 * byte)) & 0xFFu) << 5];
+// Table value of code byte `byte` of `word`: __byte_perm places that byte at
+// bits 8..15 and this lane's offset (lane_off = 4 * lane) at bits 0..7.
+__device__ __forceinline__ uint32_t lut_at(const uint8_t* lut, uint32_t lane_off, uint32_t word, int byte) {
+  return *reinterpret_cast<const uint32_t*>(lut + __byte_perm(word, lane_off, 0x7704u | (byte << 4)));
 }
 
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
@@ -242,9 +232,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ SkParams p) {
   extern __shared__ uint8_t sk_dyn[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sk_dyn) + 1023) & ~uintptr_t(1023));
+  // 1024-aligned base (swizzle atoms), kept as an offset from the shared array so
+  // that every access below compiles to a shared-memory load
+  uint8_t* smem = sk_dyn + ((1024u - (smem_u32(sk_dyn) & 1023u)) & 1023u);
   const SkLayout L = sk_layout(p.stages, p.scale_bytes);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
+  const uint8_t* lut_b = smem + L.lut;
   uint8_t* ring = smem + L.ring;
   uint8_t* sbuf = smem + L.scale;
   float* red = reinterpret_cast<float*>(smem + L.red);
@@ -252,13 +245,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   int32_t* s_off = s_chunk + (kMaxExperts + 1);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + SK_MAX_STAGES;
-  uint64_t* sfull = empty + SK_MAX_STAGES;      // [2]
-  uint64_t* sempty = sfull + 2;                 // [2]
-  uint64_t* rfull = sempty + 2;
+  uint64_t* sfull = empty + SK_MAX_STAGES;      // [SK_SBUF]
+  uint64_t* sempty = sfull + SK_SBUF;           // [SK_SBUF]
+  uint64_t* rfull = sempty + SK_SBUF;
   uint64_t* rempty = rfull + 1;
-  int32_t* s_unit = reinterpret_cast<int32_t*>(rempty + 1);   // [2]
-  int32_t* s_abort = s_unit + 2;
-  uint16_t* s_level = reinterpret_cast<uint16_t*>(smem + L.bar + 192);   // [16]
+  int32_t* s_unit = reinterpret_cast<int32_t*>(rempty + 1);   // [SK_SBUF]
+  int32_t* s_abort = s_unit + SK_SBUF;
+  uint16_t* s_level = reinterpret_cast<uint16_t*>(smem + L.bar + 224);   // [16], after barriers and unit ids
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -266,12 +259,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], SK_CONSUMERS);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < SK_SBUF; ++b) {
       mbar_init(&sfull[b], 1);
       mbar_init(&sempty[b], SK_CONSUMERS);
     }
     mbar_init(rfull, SK_CONSUMERS);
-    mbar_init(rempty, SK_CONSUMERS);
+    mbar_init(rempty, SK_CONSUMERS / 2);   // the warps that finish tiles
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -290,6 +283,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   // Byte -> bf16 pair table, one copy per lane so every lane reads its own bank.
   for (int i = threadIdx.x; i < 256 * 32; i += SK_THREADS) {
     const uint32_t b = static_cast<uint32_t>(i) >> 5;
+    const uint32_t at = b * 64 + (static_cast<uint32_t>(i) & 31u);
     uint32_t v;
     if (FMT == E4B_NF4) {   // element 2j in the high nibble -> low half
       v = static_cast<uint32_t>(s_level[b >> 4]) | (static_cast<uint32_t>(s_level[b & 15u]) << 16);
@@ -297,7 +291,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       __nv_bfloat162 t = __floats2bfloat162_rn(e2m1_value(b & 15u), e2m1_value(b >> 4));
       v = *reinterpret_cast<uint32_t*>(&t);
     }
-    lut[i] = v;
+    lut[at] = v;
   }
   __syncthreads();
 
@@ -316,42 +310,22 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         if (u >= total) drained = true;
         return u < total ? u : total;
       };
-      // packed rows of a unit: two contiguous runs; warm L2 with them two units ahead
-      auto warm = [&](int u) {
-        if (u >= total) return;
-        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
-        int row_a, row_b;
-        unit_rows<MODE>(p, un, row_a, row_b);
-        for (int half = 0; half < 2; ++half) {
-          const int row0 = half == 0 ? row_a : row_b;
-          const int nrows = min(64, p.N - row0);
-          if (nrows > 0)
-            bulk_prefetch_l2(p.codes + (static_cast<int64_t>(un.e) * p.N + row0) * (p.K / 2),
-                             static_cast<uint32_t>(nrows) * (p.K / 2));
-        }
-      };
-      int q0 = fetch(), q1 = fetch();
-      warm(q0);
-      warm(q1);
-      int sb = 0, slot = 0;
-      uint32_t sph = 0, ph = 0, armed = 0, par = 0, sarmed = 0, spar = 0;
+      uint32_t armed = 0, par = 0, sarmed = 0, spar = 0;
       bool ok = true;
-      for (;;) {
-        const int u = q0;
-        q0 = q1;
-        q1 = fetch();
-        warm(q1);
-        if (!mbar_wait(&sempty[sb], sph ^ 1u, wctx, 711)) { ok = false; break; }
+      // unit k's scale rows go to buffer k % SK_SBUF, one unit ahead of its stages
+      auto issue_scales = [&](int k, int u) -> bool {
+        const int sb = k % SK_SBUF;
+        const uint32_t sph = static_cast<uint32_t>(k / SK_SBUF) & 1u;
+        if (!mbar_wait(&sempty[sb], sph ^ 1u, wctx, 711)) return false;
         if (u >= total) {
           s_unit[sb] = -1;
           mbar_arrive(&sfull[sb]);
-          break;
+          return true;
         }
         const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
         int row_a, row_b;
         unit_rows<MODE>(p, un, row_a, row_b);
         const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
-        // the unit's scale rows (64 + 64), each half one contiguous 16-byte aligned run
         s_unit[sb] = u;
         uint8_t* sdst = sbuf + sb * p.scale_bytes;
         if (p.scale_tma) {
@@ -367,6 +341,18 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         }
         sarmed |= 1u << sb;
         spar = (spar & ~(1u << sb)) | (sph << sb);
+        return true;
+      };
+      int q0 = fetch(), q1 = fetch(), q2 = fetch();
+      int slot = 0;
+      uint32_t ph = 0;
+      int u = q0;
+      ok = issue_scales(0, u);
+      for (int k = 0; ok && u < total; ++k) {
+        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+        int row_a, row_b;
+        unit_rows<MODE>(p, un, row_a, row_b);
+        const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
         for (int st = 0; st < nst; ++st) {
           if (!mbar_wait(&empty[slot], ph ^ 1u, wctx, 712)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[slot], SK_STAGE_BYTES);
@@ -381,7 +367,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           if (++slot == p.stages) { slot = 0; ph ^= 1u; }
         }
         if (!ok) break;
-        if (++sb == 2) { sb = 0; sph ^= 1u; }
+        u = q1;
+        q1 = q2;
+        q2 = fetch();
+        ok = issue_scales(k + 1, u);
       }
       while (!drained) (void)fetch();
       // the last CTA through resets the counters for the next launch
@@ -393,16 +382,37 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       if (!ok) {   // let every issued copy land before the CTA's shared memory is released
         for (int s = 0; s < p.stages; ++s)
           if (armed & (1u << s)) mbar_drain(&full[s], (par >> s) & 1u, p.wait_limit_ns);
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < SK_SBUF; ++b)
           if (sarmed & (1u << b)) mbar_drain(&sfull[b], (spar >> b) & 1u, p.wait_limit_ns);
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int wr = warp >> 2, wk = warp & 3;
+    const int wr = warp >> 2, wk = warp & 3;   // tiles SK_TPW*wr.., 64-K block wk of each stage
     const int g = lane >> 2, c = lane & 3;
-    const uint32_t* lut_l = lut + lane;
-    const uint32_t ring_s = smem_u32(ring);
+    // fragment row g reads stage row 8t + rho (rho even for g < 4, odd for g >= 4),
+    // so the eight 16-byte chunks a half-warp loads sit in different banks
+    const int rho = 2 * (g & 3) + (g >> 2);
+    const uint32_t lane_off = 4u * lane;
+    constexpr int esz = FMT == E4B_NF4 ? 4 : 2;
+    // per-warp constant offsets: code bytes [8c, 8c+8) of block wk in rows r0, r1
+    // of each tile (128-byte swizzle), this lane's activation chunks, scale rows
+    int co[SK_TPW][2], so[SK_TPW][2];
+#pragma unroll
+    for (int j = 0; j < SK_TPW; ++j) {
+      const int t = SK_TPW * wr + j;
+      const int r[2] = {MODE == 0 ? 8 * t + rho : 16 * t + rho, MODE == 0 ? 64 + 8 * t + rho : 16 * t + 8 + rho};
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        co[j][rr] = 128 * r[rr] + 16 * ((2 * wk + (c >> 1)) ^ rho) + 8 * (c & 1);
+        so[j][rr] = r[rr] * p.srow;
+      }
+    }
+    const int xo0 = SK_CODE_BYTES + 1024 * wk + 128 * g + 16 * ((2 * c) ^ g);
+    const int xo1 = SK_CODE_BYTES + 1024 * wk + 128 * g + 16 * ((2 * c + 1) ^ g);
+    // the scale buffer's swizzle flips bits 4..6 by bits 7..9 of the row offset,
+    // which are the same for every row this lane reads
+    const uint32_t xg = (static_cast<uint32_t>(so[0][0]) >> 3) & p.scale_swz;
     int sb = 0, slot = 0;
     uint32_t sph = 0, ph = 0, rph = 0;
     bool ok = true;
@@ -411,43 +421,37 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       const int u = s_unit[sb];
       if (u < 0) break;
       const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
-      const uint32_t sc_s = smem_u32(sbuf + sb * p.scale_bytes);
-      float acc[4][4];
+      const uint8_t* scb = sbuf + sb * p.scale_bytes;
+      float acc[SK_TPW][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int j = 0; j < SK_TPW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
       for (int st = 0; st < nst; ++st) {
         if (!warp_wait(&full[slot], ph, wctx, 722)) { ok = false; break; }
         const int blk = 4 * st + wk;
         if (blk < KB) {
-          const uint32_t cs = ring_s + slot * SK_STAGE_BYTES;
-          const uint32_t xs = cs + SK_CODE_BYTES + 1024 * wk + 128 * g;
-          const uint4 xa = lds128(xs + 16 * ((2 * c) ^ g));
-          const uint4 xb = lds128(xs + 16 * ((2 * c + 1) ^ g));
+          const uint8_t* cs = ring + slot * SK_STAGE_BYTES;
+          const uint8_t* sc = scb + ((static_cast<uint32_t>(blk * esz)) ^ xg);
+          const uint4 xa = *reinterpret_cast<const uint4*>(cs + xo0);
+          const uint4 xb = *reinterpret_cast<const uint4*>(cs + xo1);
           const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-          const uint32_t half8 = 8 * (c & 1);
-          const uint32_t chunk = 2 * wk + (c >> 1);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int t = 4 * wr + j;
-            const int r0 = MODE == 0 ? 8 * t + g : 16 * t + g;
-            const int r1 = MODE == 0 ? 64 + 8 * t + g : 16 * t + 8 + g;
-            const uint2 q0 = lds64(cs + 128 * r0 + 16 * (chunk ^ g) + half8);
-            const uint2 q1 = lds64(cs + 128 * r1 + 16 * (chunk ^ g) + half8);
-            uint32_t o0 = r0 * p.srow + blk * (FMT == E4B_NF4 ? 4 : 2);
-            uint32_t o1 = r1 * p.srow + blk * (FMT == E4B_NF4 ? 4 : 2);
-            o0 ^= (o0 >> 3) & p.scale_swz;
-            o1 ^= (o1 >> 3) & p.scale_swz;
-            const uint32_t s0 = FMT == E4B_NF4 ? lds32(sc_s + o0) : lds16(sc_s + o0);
-            const uint32_t s1 = FMT == E4B_NF4 ? lds32(sc_s + o1) : lds16(sc_s + o1);
+          for (int j = 0; j < SK_TPW; ++j) {
+            const uint2 q0 = *reinterpret_cast<const uint2*>(cs + co[j][0]);
+            const uint2 q1 = *reinterpret_cast<const uint2*>(cs + co[j][1]);
+            const uint32_t s0 = FMT == E4B_NF4 ? *reinterpret_cast<const uint32_t*>(sc + so[j][0])
+                                               : *reinterpret_cast<const uint16_t*>(sc + so[j][0]);
+            const uint32_t s1 = FMT == E4B_NF4 ? *reinterpret_cast<const uint32_t*>(sc + so[j][1])
+                                               : *reinterpret_cast<const uint16_t*>(sc + so[j][1]);
             if (FMT == E4B_NF4) {
-              float bs[4] = {0.f, 0.f, 0.f, 0.f};
+              float bs[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const uint32_t w0 = i < 2 ? q0.x : q0.y, w1 = i < 2 ? q1.x : q1.y;
                 const int by = 2 * (i & 1);
-                const uint32_t a[4] = {lut_at(lut_l, w0, by), lut_at(lut_l, w1, by), lut_at(lut_l, w0, by + 1),
-                                       lut_at(lut_l, w1, by + 1)};
-                mma_bf16(bs, a, xw[2 * i], xw[2 * i + 1]);
+                const uint32_t a[4] = {lut_at(lut_b, lane_off, w0, by), lut_at(lut_b, lane_off, w1, by),
+                                       lut_at(lut_b, lane_off, w0, by + 1), lut_at(lut_b, lane_off, w1, by + 1)};
+                if (i == 0) mma_bf16_z(bs, a, xw[0], xw[1]);
+                else mma_bf16(bs, a, xw[2 * i], xw[2 * i + 1]);
               }
               const float f0 = __uint_as_float(s0), f1 = __uint_as_float(s1);
               acc[j][0] = fmaf(f0, bs[0], acc[j][0]);
@@ -461,9 +465,10 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
               for (int i = 0; i < 4; ++i) {
                 const uint32_t w0 = i < 2 ? q0.x : q0.y, w1 = i < 2 ? q1.x : q1.y;
                 const int by = 2 * (i & 1);
-                const uint32_t a[4] = {bf16x2_mul(lut_at(lut_l, w0, by), e0), bf16x2_mul(lut_at(lut_l, w1, by), e1),
-                                       bf16x2_mul(lut_at(lut_l, w0, by + 1), e0),
-                                       bf16x2_mul(lut_at(lut_l, w1, by + 1), e1)};
+                const uint32_t a[4] = {bf16x2_mul(lut_at(lut_b, lane_off, w0, by), e0),
+                                       bf16x2_mul(lut_at(lut_b, lane_off, w1, by), e1),
+                                       bf16x2_mul(lut_at(lut_b, lane_off, w0, by + 1), e0),
+                                       bf16x2_mul(lut_at(lut_b, lane_off, w1, by + 1), e1)};
                 mma_bf16(acc[j], a, xw[2 * i], xw[2 * i + 1]);
               }
             }
@@ -476,26 +481,31 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sempty[sb]);
-      // sum the four K-partials of each tile; warp (wr, wk) finishes tile 4wr+wk
+      // sum the four K-partials of each tile; warp (wr, wk < SK_TPW) finishes tile SK_TPW*wr+wk
       if (!warp_wait(rempty, rph ^ 1u, wctx, 723)) break;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < SK_TPW; ++j)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) red[((warp * 4 + j) * 4 + i) * 32 + lane] = acc[j][i];
+        for (int i = 0; i < 4; ++i) red[((warp * SK_TPW + j) * 4 + i) * 32 + lane] = acc[j][i];
       __syncwarp();
       if (lane == 0) mbar_arrive(rfull);
+      if (wk >= SK_TPW) {
+        rph ^= 1u;
+        if (++sb == SK_SBUF) { sb = 0; sph ^= 1u; }
+        continue;
+      }
       if (!warp_wait(rfull, rph, wctx, 724)) break;
       float v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] += red[(((4 * wr + k) * 4 + wk) * 4 + i) * 32 + lane];
+        for (int i = 0; i < 4; ++i) v[i] += red[(((4 * wr + k) * SK_TPW + wk) * 4 + i) * 32 + lane];
       __syncwarp();
       if (lane == 0) mbar_arrive(rempty);
       rph ^= 1u;
-      const int t = 4 * wr + wk;
+      const int t = SK_TPW * wr + wk;
       if (MODE == 0) {
-        const int col = 64 * un.nb + 8 * t + g;
+        const int col = 64 * un.nb + 8 * t + rho;
         if (p.lora_rank > 0) {
           // LoRA step: A = B_e^T (rows n, K = rank padded to 16), B = xa (scale folded in)
           uint32_t b0 = 0u, b1 = 0u;
@@ -522,7 +532,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           }
         }
       } else {
-        const int n = SK_ROWS * un.nb + 16 * t + g;
+        const int n = SK_ROWS * un.nb + 16 * t + rho;
         float* y = static_cast<float*>(p.out);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -533,7 +543,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           }
         }
       }
-      if (++sb == 2) { sb = 0; sph ^= 1u; }
+      if (++sb == SK_SBUF) { sb = 0; sph ^= 1u; }
     }
   }
 }

@@ -83,8 +83,11 @@ typedef struct {
   int32_t lora_rank;       /* 0 = no LoRA; else 1..16 */
   float lora_scale;        /* alpha / r, multiplies the LoRA delta */
   int32_t act;             /* E4B_ACT_SWIGLU */
-  int32_t tokens_per_tile; /* 0 = chosen by the library; 8 = decode kernel (warp-level MMA, codes decoded in
-                              registers, chunks of 8 tokens); else 32, 64, 128, 192 or 256 (tcgen05 tiles) */
+  int32_t tokens_per_tile; /* 0 = chosen by the library (the decode kernel when the mean number of rows
+                              per routed expert is at most 12, else a tcgen05 tile); 8 = decode kernel
+                              (codes decoded in registers, warp-level MMA, chunks of 8 tokens; needs the
+                              scale rows of 128 weight rows of both stacks to fit in shared memory, else
+                              E4B_ERR_UNSUPPORTED); 32, 64, 128, 192 or 256 = tcgen05 tile width */
 } e4b_moe_desc;
 
 /* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */
@@ -188,7 +191,9 @@ size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
  *               (both or neither, and r == d->lora_rank)
  *   out       : [T, H] bf16                            (device, written)
  *   ws        : workspace, 256-byte aligned, >= e4b_moe_workspace_bytes(d, T);
- *               its first 256 bytes hold the device status word
+ *               its first 256 bytes hold the device status word and the decode
+ *               kernel's work counters (zeroed by the route stage, left at zero
+ *               by every launch that completes)
  * bf16 outputs match the fp64 definition within relative Frobenius error
  * 5e-3 and max-abs error 3e-2 * max|ref|; routing is bit-exact.
  */

@@ -61,8 +61,13 @@ def test_forward_validation_and_workspace(L):
     for bad in [e4b.make_desc(8, 250, 128, 2, "mxfp4"), e4b.make_desc(8, 256, 100, 2, "mxfp4"),
                 e4b.make_desc(8, 256, 128, 9, "mxfp4"), e4b.make_desc(300, 256, 128, 2, "nf4"),
                 e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=17),
-                e4b.make_desc(8, 256, 128, 2, "nf4", tokens_per_tile=48)]:
+                e4b.make_desc(8, 256, 128, 2, "nf4", tokens_per_tile=48),
+                # decode kernel asked for, but 128 rows of 8192/64 fp32 scales per unit do not fit
+                e4b.make_desc(8, 8192, 128, 2, "nf4", tokens_per_tile=8)]:
         assert e4b.e4b_moe_workspace_bytes(bad, 64) == 0
+    # the same shape is served by the tcgen05 tiles, and by the decode kernel at 2048
+    assert e4b.e4b_moe_workspace_bytes(e4b.make_desc(8, 8192, 128, 2, "nf4"), 64) > 0
+    assert e4b.e4b_moe_workspace_bytes(e4b.make_desc(8, 2048, 128, 2, "nf4", tokens_per_tile=8), 64) > 0
     # one-sided LoRA is refused before any launch
     dl = e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=8, lora_scale=2.0)
     st = L.e4b_moe_forward(ctypes.byref(dl), 4, None, None, None, None, None, None, 256, None, None, 256,

@@ -36,7 +36,7 @@ def test_tiny_layer_routing_intermediates_bit_exact():
     assert np.array_equal(xs, x[r["sorted_slot"] // TINY.k])
 
 
-@pytest.mark.parametrize("tpt", [0, 8])
+@pytest.mark.parametrize("tpt", [0, 8, 32])
 @pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
 @pytest.mark.parametrize("T", [1, 3, 200])
 def test_small_layers_ragged(fmt, T, tpt):
@@ -76,7 +76,7 @@ def test_lora_tiny_and_zero_b(fmt, tpt):
     assert not torch.equal(out_l.view(torch.int16), out_b.view(torch.int16))
 
 
-@pytest.mark.parametrize("tpt", [0, 8])
+@pytest.mark.parametrize("tpt", [0, 32])
 @pytest.mark.parametrize("T", [1, 8])
 def test_qwen3_nf4_decode_full(T, tpt):
     run_and_compare(QWEN, T, tokens_per_tile=tpt)
