@@ -262,6 +262,9 @@ def bench_e4b(args, world, rank, local):
     g_fwd = capture(forward)
     g_gu = capture(lambda: stage(e4b.E4B_STAGE_GATE_UP))
     g_dn = capture(lambda: stage(e4b.E4B_STAGE_DOWN))
+    g_small = {nm: capture(lambda st=st: stage(st)) for nm, st in
+               (("route_ms", e4b.E4B_STAGE_ROUTE), ("gather_ms", e4b.E4B_STAGE_GATHER),
+                ("combine_ms", e4b.E4B_STAGE_COMBINE))}
     for _ in range(3):
         g_fwd.replay()
     torch.cuda.synchronize()
@@ -297,9 +300,10 @@ def bench_e4b(args, world, rank, local):
     # the dominant kernel, launch by launch (touched weights per launch exceed L2: no flush needed)
     gu_ms = max_over_ranks(time_graph(g_gu, K))
     dn_ms = max_over_ranks(time_graph(g_dn, K))
+    small_ms = {nm: max_over_ranks(time_graph(g, K)) for nm, g in g_small.items()}
     if e4b.e4b_device_status(ws) != e4b.E4B_OK:
         raise RuntimeError("device status reported an error in the timed region")
-    del g_fwd, g_gu, g_dn
+    del g_fwd, g_gu, g_dn, g_small
 
     # end to end through the public call with host buffers: H2D inputs, forward, D2H output, every step
     x_h = torch.from_numpy(x_np.view(np.int16)).pin_memory()
@@ -346,7 +350,7 @@ def bench_e4b(args, world, rank, local):
                      "frac": achieved / peaks["hbm_gbs"], "peak_kind": peak_kind,
                      "traffic": recorded_traffic("gate_up"),
                      "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms},
-        "kernels": {"gate_up_ms": gu_ms, "down_ms": dn_ms,
+        "kernels": {"gate_up_ms": gu_ms, "down_ms": dn_ms, **small_ms,
                     "down_gbs": dn_bytes / (dn_ms * 1e-3) / 1e9,
                     "layer_weight_gbs": layer_weight_bytes / (ms_per_step * 1e-3) / 1e9,
                     "touched_experts": touched},

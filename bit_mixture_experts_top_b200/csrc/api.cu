@@ -185,7 +185,6 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, in
   const RouteLayout L = route_layout(T, E, k);
   if (ws_bytes < L.total) return E4B_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) return E4B_ERR_CUDA;
   RouteBuffers b;
   b.status = at<int32_t>(ws, L.status);
   b.done_counter = reinterpret_cast<uint32_t*>(b.status + 2);
@@ -196,7 +195,8 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, in
   b.block_counts = at<int32_t>(ws, L.block_counts);
   b.sorted_slot = sorted_slot;
   b.slot_pos = at<int32_t>(ws, L.slot_pos);
-  return launch_route(logits, T, E, k, 0, b, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  // the status words are zeroed by the launch sequence (in-kernel for one routing block)
+  return launch_route(logits, T, E, k, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }
 
 size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T) {
@@ -276,8 +276,8 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   for (int32_t stage = first; stage <= last; ++stage) {
     switch (stage) {
       case E4B_STAGE_ROUTE:
-        if (cudaMemsetAsync(ws, 0, kStatusBytes, s) != cudaSuccess) return E4B_ERR_CUDA;
-        if (launch_route(logits, T, d->E, d->k, tpt, b, s) != cudaSuccess) return E4B_ERR_CUDA;
+        // zeroes the status words first (in the routing kernel when one block routes)
+        if (launch_route(logits, T, d->E, d->k, tpt, b, b.status, s) != cudaSuccess) return E4B_ERR_CUDA;
         break;
       case E4B_STAGE_GATHER:
         if (launch_gather(x, d->H, d->k, R, b.sorted_slot, b.topk_ids, d->E, x_sorted, lora_A, d->lora_rank,

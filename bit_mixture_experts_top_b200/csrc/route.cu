@@ -26,6 +26,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kTopkThreads = 1024;         // top-k: 4 tokens per warp at 128 tokens per block
+constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTokPerWarp = kRouteTokensPerBlock / kTopkWarps;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ uint32_t route_key(uint16_t bits, int e) {
@@ -39,9 +42,11 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as
 // Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
 // slots of the block with the same expert).  Each warp owns a contiguous
 // segment; per-warp histograms are scanned across warps first.
+template <int NW>
 __device__ __forceinline__ void rank_block(int b, const int32_t* __restrict__ topk_ids, int T, int E, int k,
                                            const int32_t* block_base, int32_t* __restrict__ sorted_slot,
                                            int32_t* __restrict__ slot_pos, int32_t (*s_wc)[kMaxExperts]) {
+  constexpr int kWarps = NW, kThreads = NW * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t s0 = static_cast<int64_t>(b) * kRouteTokensPerBlock * k;
   const int64_t s1 = min(static_cast<int64_t>(T), static_cast<int64_t>(b + 1) * kRouteTokensPerBlock) * k;
@@ -85,53 +90,60 @@ __global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __r
                                                               int32_t* __restrict__ sorted_slot,
                                                               int32_t* __restrict__ slot_pos) {
   __shared__ int32_t s_wc[kWarps][kMaxExperts];
-  rank_block(blockIdx.x, topk_ids, T, E, k, block_base, sorted_slot, slot_pos, s_wc);
+  rank_block<kWarps>(blockIdx.x, topk_ids, T, E, k, block_base, sorted_slot, slot_pos, s_wc);
 }
 
-__global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E, int k,
-                                                              int tokens_per_tile, int nblk,
-                                                              int32_t* __restrict__ topk_ids,
-                                                              float* __restrict__ topk_w, int32_t* block_counts,
-                                                              uint32_t* done_counter, int32_t* expert_offsets,
-                                                              int32_t* chunk_off, int32_t* __restrict__ sorted_slot,
-                                                              int32_t* __restrict__ slot_pos) {
-  __shared__ int32_t s_wc[kWarps][kMaxExperts];
+__global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E,
+                                                                  int k, int tokens_per_tile, int nblk,
+                                                                  int32_t* __restrict__ topk_ids,
+                                                                  float* __restrict__ topk_w, int32_t* block_counts,
+                                                                  uint32_t* done_counter, int32_t* expert_offsets,
+                                                                  int32_t* chunk_off, int32_t* __restrict__ sorted_slot,
+                                                                  int32_t* __restrict__ slot_pos) {
+  __shared__ int32_t s_wc[kTopkWarps][kMaxExperts];
   __shared__ int32_t s_cnt[kMaxExperts];
   __shared__ int32_t s_tot[kMaxExperts + 1];
   __shared__ bool s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < E; e += kThreads) s_cnt[e] = 0;
+  for (int e = tid; e < E; e += kTopkThreads) s_cnt[e] = 0;
   __syncthreads();
 
+  // warp w takes tokens t_begin + w + kTopkWarps * q; all their logits are loaded first
   const int t_begin = blockIdx.x * kRouteTokensPerBlock;
   const int per_lane = (E + 31) >> 5;      // <= 8
-  for (int tt = warp; tt < kRouteTokensPerBlock; tt += kWarps) {
-    const int t = t_begin + tt;
-    if (t >= T) break;
+  uint32_t key[kTokPerWarp][kMaxExperts / 32];
+#pragma unroll
+  for (int q = 0; q < kTokPerWarp; ++q) {
+    const int t = t_begin + warp + kTopkWarps * q;
     const uint16_t* row = logits + static_cast<int64_t>(t) * E;
-    uint32_t key[kMaxExperts / 32];
 #pragma unroll
     for (int j = 0; j < kMaxExperts / 32; ++j) {
       const int e = lane + 32 * j;
-      key[j] = (j < per_lane && e < E) ? route_key(row[e], e) : 0u;   // real keys are never 0
+      key[q][j] = (t < T && j < per_lane && e < E) ? route_key(__ldg(row + e), e) : 0u;   // real keys are never 0
     }
+  }
+#pragma unroll
+  for (int q = 0; q < kTokPerWarp; ++q) {
+    const int t = t_begin + warp + kTopkWarps * q;
+    if (t >= T) break;
     uint32_t mine = 0;                     // lane j keeps the j-th pick
     for (int r = 0; r < k; ++r) {
       uint32_t best = 0;
 #pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[j]);
+      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
       best = __reduce_max_sync(kFull, best);
       const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
 #pragma unroll
       for (int j = 0; j < kMaxExperts / 32; ++j)
-        if (lane + 32 * j == e) key[j] = 0u;
+        if (lane + 32 * j == e) key[q][j] = 0u;
       if (lane == r) mine = best;
     }
     int id = 0;
     float v = 0.0f;
     if (lane < k) {
       id = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
-      v = bf16_bits_to_f32(row[id]);
+      const uint32_t ord = mine >> 16;     // invert route_key: the bf16 bits of the pick
+      v = bf16_bits_to_f32(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu)));
     }
     const float m = __shfl_sync(kFull, v, 0);          // the first pick holds the maximum
     float ex = (lane < k) ? expf(v - m) : 0.0f;
@@ -145,7 +157,7 @@ __global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __
     }
   }
   __syncthreads();
-  for (int e = tid; e < E; e += kThreads) block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = s_cnt[e];
+  for (int e = tid; e < E; e += kTopkThreads) block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = s_cnt[e];
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(done_counter, 1u) == static_cast<uint32_t>(nblk - 1));
@@ -154,28 +166,52 @@ __global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __
 
   // Last block: totals, exclusive offsets, per-block bases, tile-chunk offsets.
   __threadfence();
-  for (int e = tid; e < E; e += kThreads) {
+  for (int e = tid; e < E; e += kTopkThreads) {
     int32_t tot = 0;
     for (int b = 0; b < nblk; ++b) tot += __ldcg(block_counts + static_cast<int64_t>(b) * E + e);
     s_tot[e] = tot;
   }
   __syncthreads();
-  if (tid == 0) {
+  if (warp == 0) {
+    // warp-wide exclusive scans of the counts and of the chunk counts; lane l owns
+    // experts [8l, 8l+8)
+    int32_t c[kMaxExperts / 32], ch[kMaxExperts / 32];
     int32_t run = 0, crun = 0;
-    for (int e = 0; e < E; ++e) {
-      const int32_t c = s_tot[e];
-      expert_offsets[e] = run;
-      if (chunk_off) chunk_off[e] = crun;
-      s_tot[e] = run;
-      run += c;
-      if (tokens_per_tile > 0) crun += (c + tokens_per_tile - 1) / tokens_per_tile;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane * (kMaxExperts / 32) + j;
+      c[j] = e < E ? s_tot[e] : 0;
+      ch[j] = tokens_per_tile > 0 ? (c[j] + tokens_per_tile - 1) / tokens_per_tile : 0;
+      run += c[j];
+      crun += ch[j];
     }
-    expert_offsets[E] = run;
-    if (chunk_off) chunk_off[E] = crun;
-    *done_counter = 0u;                               // ready for the next call
+    int32_t inc = run, cinc = crun;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t a = __shfl_up_sync(kFull, inc, off), ca = __shfl_up_sync(kFull, cinc, off);
+      if (lane >= off) { inc += a; cinc += ca; }
+    }
+    run = inc - run;
+    crun = cinc - crun;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane * (kMaxExperts / 32) + j;
+      if (e < E) {
+        expert_offsets[e] = run;
+        if (chunk_off) chunk_off[e] = crun;
+        s_tot[e] = run;
+      }
+      run += c[j];
+      crun += ch[j];
+    }
+    if (lane == 31) {
+      expert_offsets[E] = run;
+      if (chunk_off) chunk_off[E] = crun;
+      *done_counter = 0u;                             // ready for the next call
+    }
   }
   __syncthreads();
-  for (int e = tid; e < E; e += kThreads) {
+  for (int e = tid; e < E; e += kTopkThreads) {
     int32_t run = s_tot[e];
     for (int b = 0; b < nblk; ++b) {
       int32_t* p = block_counts + static_cast<int64_t>(b) * E + e;
@@ -187,7 +223,150 @@ __global__ void __launch_bounds__(kThreads) route_topk_kernel(const uint16_t* __
   if (nblk == 1) {          // a single routing block also ranks its slots: one launch for small batches
     __threadfence_block();
     __syncthreads();
-    rank_block(0, topk_ids, T, E, k, block_counts, sorted_slot, slot_pos, s_wc);
+    rank_block<kTopkWarps>(0, topk_ids, T, E, k, block_counts, sorted_slot, slot_pos, s_wc);
+  }
+}
+
+// T <= 128 (one routing block): top-k, histogram, scans and the stable rank in
+// one block with every intermediate in shared memory, no cross-block protocol.
+// The block also zeroes the status words of the workspace first (the caller
+// skips its memset), so a small forward starts with a single launch.
+__global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
+                                                                  int k, int tokens_per_tile, int32_t* status_words,
+                                                                  int32_t* __restrict__ topk_ids,
+                                                                  float* __restrict__ topk_w,
+                                                                  int32_t* __restrict__ expert_offsets,
+                                                                  int32_t* __restrict__ chunk_off,
+                                                                  int32_t* __restrict__ sorted_slot,
+                                                                  int32_t* __restrict__ slot_pos) {
+  __shared__ int16_t s_ids[kRouteTokensPerBlock * kMaxTopK];
+  __shared__ __align__(16) int16_t s_wc[kTopkWarps][kMaxExperts];   // per-warp counts, then running positions
+  __shared__ int32_t s_cnt[kMaxExperts];
+  __shared__ int32_t s_off[kMaxExperts];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (status_words && tid < kStatusBytes / 4) status_words[tid] = 0;
+  for (int e = tid; e < kMaxExperts; e += kTopkThreads) s_cnt[e] = 0;
+  for (int i = tid; i < kTopkWarps * kMaxExperts; i += kTopkThreads) (&s_wc[0][0])[i] = 0;
+  __syncthreads();
+
+  const int per_lane = (E + 31) >> 5;
+  uint32_t key[kTokPerWarp][kMaxExperts / 32];
+#pragma unroll
+  for (int q = 0; q < kTokPerWarp; ++q) {
+    const int t = warp + kTopkWarps * q;
+    const uint16_t* row = logits + static_cast<int64_t>(t) * E;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane + 32 * j;
+      key[q][j] = (t < T && j < per_lane && e < E) ? route_key(__ldg(row + e), e) : 0u;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kTokPerWarp; ++q) {
+    const int t = warp + kTopkWarps * q;
+    if (t >= T) break;
+    uint32_t mine = 0;
+    for (int r = 0; r < k; ++r) {
+      uint32_t best = 0;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
+      best = __reduce_max_sync(kFull, best);
+      const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j)
+        if (lane + 32 * j == e) key[q][j] = 0u;
+      if (lane == r) mine = best;
+    }
+    int id = 0;
+    float v = 0.0f;
+    if (lane < k) {
+      id = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
+      const uint32_t ord = mine >> 16;
+      v = bf16_bits_to_f32(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu)));
+    }
+    const float m = __shfl_sync(kFull, v, 0);
+    float ex = (lane < k) ? expf(v - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    if (lane < k) {
+      topk_ids[static_cast<int64_t>(t) * k + lane] = id;
+      topk_w[static_cast<int64_t>(t) * k + lane] = ex / sum;
+      s_ids[t * k + lane] = static_cast<int16_t>(id);
+      atomicAdd(&s_cnt[id], 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {          // exclusive scans of the counts and chunk counts; lane l owns experts [8l, 8l+8)
+    int32_t c[kMaxExperts / 32], ch[kMaxExperts / 32];
+    int32_t run = 0, crun = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane * (kMaxExperts / 32) + j;
+      c[j] = e < E ? s_cnt[e] : 0;
+      ch[j] = tokens_per_tile > 0 ? (c[j] + tokens_per_tile - 1) / tokens_per_tile : 0;
+      run += c[j];
+      crun += ch[j];
+    }
+    int32_t inc = run, cinc = crun;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t a = __shfl_up_sync(kFull, inc, off), ca = __shfl_up_sync(kFull, cinc, off);
+      if (lane >= off) { inc += a; cinc += ca; }
+    }
+    run = inc - run;
+    crun = cinc - crun;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane * (kMaxExperts / 32) + j;
+      if (e < E) {
+        expert_offsets[e] = run;
+        if (chunk_off) chunk_off[e] = crun;
+        s_off[e] = run;
+      }
+      run += c[j];
+      crun += ch[j];
+    }
+    if (lane == 31) {
+      expert_offsets[E] = run;
+      if (chunk_off) chunk_off[E] = crun;
+    }
+  }
+  // stable rank: warp w owns the contiguous slot segment [w0, w1)
+  const int n = T * k;
+  const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+  const int w0 = warp * seg, w1 = min(n, w0 + seg);
+  for (int s = w0 + lane; s < w1; s += 32) {
+    const int id = s_ids[s];
+    // 16-bit counters: add through the containing word
+    atomicAdd(reinterpret_cast<int*>(&s_wc[warp][id & ~1]), 1 << (16 * (id & 1)));
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kTopkThreads) {
+    int32_t run = s_off[e];
+    for (int w = 0; w < kTopkWarps; ++w) {
+      const int32_t c = s_wc[w][e];
+      s_wc[w][e] = static_cast<int16_t>(run);
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int c0 = w0; c0 < w1; c0 += 32) {
+    const int s = c0 + lane;
+    const bool valid = s < w1;
+    const int id = valid ? s_ids[s] : (kMaxExperts + lane);
+    const uint32_t peers = __match_any_sync(kFull, id);
+    const int rank = __popc(peers & lt);
+    int32_t pos = 0;
+    if (valid) pos = static_cast<uint16_t>(s_wc[warp][id]) + rank;
+    __syncwarp();
+    if (valid && rank == __popc(peers) - 1) s_wc[warp][id] = static_cast<int16_t>(pos + 1);
+    __syncwarp();
+    if (valid) {
+      sorted_slot[pos] = s;
+      slot_pos[s] = pos;
+    }
   }
 }
 
@@ -210,6 +389,18 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __rest
   float acc[kMaxLoraRank];
 #pragma unroll
   for (int j = 0; j < kMaxLoraRank; ++j) acc[j] = 0.0f;
+  if (!lora_A) {            // plain copy: eight 16-byte loads in flight per lane
+    for (int v0 = lane; v0 < nvec; v0 += 32 * 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (v0 + 32 * i < nvec) q[i] = __ldg(src + v0 + 32 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (v0 + 32 * i < nvec) dst[v0 + 32 * i] = q[i];
+    }
+    return;
+  }
   const uint16_t* Ae = lora_A ? lora_A + static_cast<int64_t>(topk_ids[slot]) * H * rank : nullptr;
   const bool vec8 = Ae && (rank == 8 || rank == 16) &&            // A rows are whole 16-byte vectors
                     (reinterpret_cast<uintptr_t>(lora_A) & 15u) == 0;
@@ -259,41 +450,62 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __rest
   reinterpret_cast<uint32_t*>(xa + r * 64)[lane] = *reinterpret_cast<uint32_t*>(&pr);
 }
 
-// One block per token: out[t] = sum_j w[t, j] * y[slot_pos[t*k + j]], j ascending.
+// out[t] = sum_j w[t, j] * y[slot_pos[t*k + j]], j ascending.  Block (t, cb)
+// covers columns [4 * kThreads * cb, ...) of token t, one float4 per thread;
+// the k rows are loaded eight at a time before they are summed in order.
 __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restrict__ y,
                                                            const float* __restrict__ topk_w,
                                                            const int32_t* __restrict__ slot_pos, int k, int H,
                                                            uint16_t* __restrict__ out) {
   const int64_t t = blockIdx.x;
-  const int nq = H / 4;
-  for (int c = threadIdx.x; c < nq; c += kThreads) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float w = __ldg(topk_w + t * k + j);
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(y + static_cast<int64_t>(__ldg(slot_pos + t * k + j)) * H) + c);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+  const int c = blockIdx.y * kThreads + threadIdx.x;
+  if (c >= H / 4) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    float4 v[8];
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (j0 + i < k) {
+        w[i] = __ldg(topk_w + t * k + j0 + i);
+        v[i] = __ldcs(reinterpret_cast<const float4*>(y + static_cast<int64_t>(__ldg(slot_pos + t * k + j0 + i)) * H) + c);
+      }
     }
-    __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 o = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
-    reinterpret_cast<uint2*>(out + t * H)[c] = o;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (j0 + i < k) {
+        acc.x = fmaf(w[i], v[i].x, acc.x);
+        acc.y = fmaf(w[i], v[i].y, acc.y);
+        acc.z = fmaf(w[i], v[i].z, acc.z);
+        acc.w = fmaf(w[i], v[i].w, acc.w);
+      }
+    }
   }
+  __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 o = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+  reinterpret_cast<uint2*>(out + t * H)[c] = o;
 }
 
 }  // namespace
 
 cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t tokens_per_tile,
-                         const RouteBuffers& b, cudaStream_t s) {
+                         const RouteBuffers& b, int32_t* status_words, cudaStream_t s) {
   if (T == 0) {
-    cudaError_t err = cudaMemsetAsync(b.expert_offsets, 0, sizeof(int32_t) * (E + 1), s);
+    cudaError_t err = status_words ? cudaMemsetAsync(status_words, 0, kStatusBytes, s) : cudaSuccess;
+    if (err == cudaSuccess) err = cudaMemsetAsync(b.expert_offsets, 0, sizeof(int32_t) * (E + 1), s);
     if (err == cudaSuccess && b.chunk_off) err = cudaMemsetAsync(b.chunk_off, 0, sizeof(int32_t) * (E + 1), s);
     return err;
   }
   const int nblk = route_blocks(T);
-  route_topk_kernel<<<nblk, kThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
+  if (nblk == 1) {
+    route_small_kernel<<<1, kTopkThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, status_words, b.topk_ids,
+                                                  b.topk_w, b.expert_offsets, b.chunk_off, b.sorted_slot,
+                                                  b.slot_pos);
+    return cudaGetLastError();
+  }
+  if (status_words && cudaMemsetAsync(status_words, 0, kStatusBytes, s) != cudaSuccess) return cudaGetLastError();
+  route_topk_kernel<<<nblk, kTopkThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
                                                b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off,
                                                b.sorted_slot, b.slot_pos);
   cudaError_t err = cudaGetLastError();
@@ -316,7 +528,8 @@ cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, co
 cudaError_t launch_combine(const float* y, const float* topk_w, const int32_t* slot_pos, int32_t T, int32_t k,
                            int32_t H, uint16_t* out, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  combine_kernel<<<T, kThreads, 0, s>>>(y, topk_w, slot_pos, k, H, out);
+  const dim3 grid(T, (H / 4 + kThreads - 1) / kThreads);
+  combine_kernel<<<grid, kThreads, 0, s>>>(y, topk_w, slot_pos, k, H, out);
   return cudaGetLastError();
 }
 
@@ -394,5 +607,5 @@ extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32
   b.block_counts = reinterpret_cast<int32_t*>(scratch + off_counts);
   b.sorted_slot = sorted_slot;
   b.slot_pos = reinterpret_cast<int32_t*>(scratch + off_pos);
-  return launch_route(logits, T, E, k, 0, b, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  return launch_route(logits, T, E, k, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }
