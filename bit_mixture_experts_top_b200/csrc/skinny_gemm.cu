@@ -25,17 +25,19 @@
 //  * mode 1 (down): output rows 128nb..128nb+127; tile t = rows 16t..16t+15.
 //
 // Warp roles (one CTA per SM, persistent):
-//  * warp 16, lane 0, the producer: takes units from a global counter (dynamic,
+//  * warp 8, lane 0, the producer: takes units from a global counter (dynamic,
 //    so every CTA finishes within one unit of the others), copies each unit's
 //    scale rows to a shared buffer one unit ahead (2 buffers; a TMA box with the hardware
 //    swizzle when a scale row is 32, 64 or 128 bytes, else one bulk copy per
 //    contiguous run) and issues the 256-K stages: 128 rows x 128 code bytes
 //    (128-byte swizzle) and the chunk's 8 activation rows x 256 K;
-//  * warps 0-15, consumers: warp (wr, wk) owns MMA tiles 2wr, 2wr+1 (32 rows)
+//  * warps 0-7, consumers: warp (wr, wk) owns MMA tiles 4wr..4wr+3 (64 rows)
 //    and the 64-K block wk of every stage, so the activation fragments it
-//    loads serve 32 rows.  At the end of a unit the four K-partials of each
-//    tile are summed through shared memory and warp (wr, wk < 2) finishes
-//    tile 2wr+wk (LoRA step, SwiGLU or the fp32 store).
+//    loads serve 64 rows (shared-memory bandwidth is the scarce resource:
+//    per 16 KB stage the byte table takes 512 wavefronts, codes 128, TMA
+//    writes 160, activations 64, scales 64).  At the end of a unit the four
+//    K-partials of each tile are summed through shared memory and warp
+//    (wr, wk) finishes tile 4wr+wk (LoRA step, SwiGLU or the fp32 store).
 //
 // Fragment/byte mapping.  Lane (g = lane / 4, c = lane % 4) takes, per 64-K
 // block, code bytes [8c, 8c+8) of fragment rows g and g+8 of a tile (fragment
@@ -61,10 +63,10 @@
 namespace e4b {
 namespace {
 
-constexpr int SK_CONSUMERS = 16;
-constexpr int SK_PRODUCER = 16;                  // warp index
-constexpr int SK_THREADS = 17 * 32;
-constexpr int SK_TPW = 2;                        // MMA tiles per consumer warp
+constexpr int SK_CONSUMERS = 8;
+constexpr int SK_PRODUCER = 8;                   // warp index
+constexpr int SK_THREADS = 9 * 32;
+constexpr int SK_TPW = 4;                        // MMA tiles per consumer warp
 constexpr int SK_SBUF = 2;                       // per-unit scale buffers
 constexpr int SK_TOK = 8;                        // tokens per chunk (MMA N)
 constexpr int SK_ROWS = 128;                     // weight rows per unit
@@ -264,7 +266,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       mbar_init(&sempty[b], SK_CONSUMERS);
     }
     mbar_init(rfull, SK_CONSUMERS);
-    mbar_init(rempty, SK_CONSUMERS / 2);   // the warps that finish tiles
+    mbar_init(rempty, (SK_CONSUMERS / 4) * SK_TPW);   // the warps that finish tiles
     *s_abort = 0;
     fence_mbar_init();
   }
