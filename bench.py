@@ -55,15 +55,16 @@ def source_digest():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_tag):
-    """DRAM bytes per launch of the kernel from the committed ncu summary, if it still matches the source."""
+def recorded_traffic(kernel_tag, workload):
+    """DRAM bytes per launch of the kernel from the committed ncu summary, if it still matches the source
+    and was taken on this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_tag)
-    if not e or e.get("source_digest") != source_digest():
+    if not e or e.get("source_digest") != source_digest() or not e.get("workload", "").startswith(workload + " "):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -218,8 +219,8 @@ def bench_e4b(args, world, rank, local):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         return float(t.item())
 
-    w = WORKLOADS[WORKLOAD]
-    T = T_HEADLINE
+    w = WORKLOADS[args.workload]
+    T = args.tokens
     lay = layer.synthetic_layer(w, dev)
     x_np, lg_np = layer.synthetic_tokens(w, T)
     x = layer.bits_tensor(x_np, dev)
@@ -334,22 +335,34 @@ def bench_e4b(args, world, rank, local):
     barrier()
 
     peaks, peak_kind = load_peaks()
-    achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
+    # the library's kernel choice (tokens_per_tile 0): the decode kernel at <= 12 rows per routed expert
+    active = min(R, w.E)
+    decode_kernel = (R + active - 1) // active <= 12
+    # decode shapes are bound by the weight stream, prefill shapes by the tensor cores
+    gu_flops = 2 * R * w.H * 2 * w.I + (2 * R * (w.H + 2 * w.I) * w.lora_rank if w.lora_rank else 0)
+    tensor_bound = gu_flops / gu_bytes > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        roof = {"bound": "tensor", "achieved": gu_flops / (gu_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "algorithmic_flops_per_launch": gu_flops}
+    else:
+        roof = {"bound": "hbm", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "algorithmic_bytes_per_launch": gu_bytes}
+    roof["frac"] = roof["achieved"] / roof["peak"]
     value = world * T / (ms_per_step * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD} T={T}", "E": w.E, "H": w.H, "I": w.I, "k": w.k, "format": w.fmt,
+        "config": {"workload": f"{args.workload} T={T}", "E": w.E, "H": w.H, "I": w.I, "k": w.k, "format": w.fmt,
                    "global_batch": T * world, "tokens_per_gpu": T, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {layer_weight_bytes / 1e6:.0f} MB of touched expert weights "
                          f"per step vs {L2_BYTES / 1e6:.0f} MB L2, no flush"},
-        "roofline": {"bound": "hbm", "kernel": "skinny_gemm gate_up (decode kernel: NF4 codes decoded in registers, "
-                                                "warp-level MMA, SwiGLU)",
-                     "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "peak_kind": peak_kind,
-                     "traffic": recorded_traffic("gate_up"),
-                     "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_ms": gu_ms},
+        "roofline": {"kernel": ("skinny_gemm gate_up (decode kernel: codes decoded in registers, warp-level MMA, "
+                                "SwiGLU)" if decode_kernel else
+                                "grouped_gemm gate_up (tcgen05, dequant to tensor memory, SwiGLU)"),
+                     **roof, "peak_kind": peak_kind,
+                     "traffic": recorded_traffic("gate_up", f"{args.workload} T={T}"),
+                     "avg_launch_ms": gu_ms},
         "kernels": {"gate_up_ms": gu_ms, "down_ms": dn_ms, **small_ms,
                     "down_gbs": dn_bytes / (dn_ms * 1e-3) / 1e9,
                     "layer_weight_gbs": layer_weight_bytes / (ms_per_step * 1e-3) / 1e9,
@@ -361,9 +374,11 @@ def bench_e4b(args, world, rank, local):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, dt, ne = oracle_tokens_per_s(w, x_np, lg_np, np.arange(T), reps=2)
+        ns = min(T, 64)     # a bounded sample of the batch for prefill shapes
+        tps, dt, ne = oracle_tokens_per_s(w, x_np, lg_np, np.arange(ns), reps=2)
+        what = f"the whole T={T} batch" if ns == T else f"the first {ns} of the T={T} tokens"
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                "sample": f"the whole T={T} batch ({ne} experts decoded in fp64), "
+                                "sample": f"{what} ({ne} experts decoded in fp64), "
                                           f"timed twice, {dt:.1f} s per forward"}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -373,13 +388,19 @@ def bench_e4b(args, world, rank, local):
 
 
 def main():
+    from bit_mixture_experts_top_b200.workloads import WORKLOADS
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD,
+                    help="synthetic layer to time (default: the headline decode workload)")
+    ap.add_argument("--tokens", type=int, default=None, help="tokens per step (default: the workload's largest)")
     args = ap.parse_args()
+    if args.tokens is None:
+        args.tokens = T_HEADLINE if args.workload == WORKLOAD else WORKLOADS[args.workload].tokens[-1]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world, rank, local = init_dist()
