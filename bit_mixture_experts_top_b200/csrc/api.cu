@@ -104,19 +104,29 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   return E4B_OK;
 }
 
-int32_t pick_tokens_per_tile(const e4b_moe_desc& d, int32_t T) {
-  if (d.tokens_per_tile) return d.tokens_per_tile;
+struct KernelChoice {
+  bool decode;        // skinny_gemm (decode kernel) or grouped_gemm (tcgen05 tiles)
+  int32_t tokens;     // decode: tokens per chunk; tcgen05: tile width
+};
+
+// Mean routed rows per active expert decides: a handful per expert -> the decode
+// kernel (weight-stream bound), with chunks of 8, 16 or 32 tokens so that one
+// decoded weight fragment serves up to 32 tokens; more -> the smallest tcgen05
+// tile that holds most experts' rows in one chunk (192, not 256, for prefill
+// keeps the weight tile in tensor memory).
+KernelChoice pick_kernel(const e4b_moe_desc& d, int32_t T) {
   const int64_t R = static_cast<int64_t>(T) * d.k;
   const int64_t active = R < d.E ? R : d.E;
   const int64_t avg = active > 0 ? (R + active - 1) / active : 1;
-  // a handful of rows per expert: the decode kernel (weight stream bound);
-  // else the smallest tcgen05 tile that holds most experts' rows in one chunk,
-  // 192 (not 256) for prefill keeps the weight tile in tensor memory
-  if (avg <= 12 && skinny_gemm_supported(d.H, d.format) && skinny_gemm_supported(d.I, d.format)) return 8;
-  if (avg <= 16) return 32;
-  if (avg <= 48) return 64;
-  if (avg <= 96) return 128;
-  return 192;
+  const bool decode_ok = skinny_gemm_supported(d.H, d.format) && skinny_gemm_supported(d.I, d.format);
+  const int32_t chunk = avg <= 8 ? 8 : (avg <= 16 ? 16 : 32);
+  if (d.tokens_per_tile == 8) return {true, chunk};
+  if (d.tokens_per_tile) return {false, d.tokens_per_tile};
+  if (avg <= kDecodeMaxRows && decode_ok) return {true, chunk};
+  if (avg <= 16) return {false, 32};
+  if (avg <= 48) return {false, 64};
+  if (avg <= 96) return {false, 128};
+  return {false, 192};
 }
 
 template <typename T>
@@ -244,7 +254,8 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
     if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 2))) return E4B_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int32_t tpt = pick_tokens_per_tile(*d, T);
+  const KernelChoice kc = pick_kernel(*d, T);
+  const int32_t tpt = kc.tokens;
   const int32_t R = T * d->k;
 
   RouteBuffers b;
@@ -268,6 +279,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   g.I = d->I;
   g.R = R;
   g.tokens_per_tile = tpt;
+  g.decode = kc.decode ? 1 : 0;
   g.expert_offsets = b.expert_offsets;
   g.chunk_off = b.chunk_off;
   g.status = b.status;
@@ -295,7 +307,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_B = lora_B;
         g.lora_rank = d->lora_rank;
         g.out = h;
-        const e4b_status st = tpt == 8 ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
+        const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
       }
@@ -310,7 +322,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_B = nullptr;
         g.lora_rank = 0;
         g.out = y;
-        const e4b_status st = tpt == 8 ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
+        const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
       }

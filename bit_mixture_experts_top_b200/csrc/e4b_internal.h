@@ -15,6 +15,7 @@ constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxLoraRank = 16;
 constexpr int kRouteTokensPerBlock = 128;   // tokens per histogram block of the router
+constexpr int kDecodeMaxRows = 12;         // auto choice: decode kernel up to this mean rows per expert
 constexpr int kStatusBytes = 256;           // status word + router done-counter at the start of a workspace
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // bounded device waits: 2 s
 
@@ -71,7 +72,8 @@ struct GroupedGemmLaunch {
   int32_t fmt;              // E4B_NF4 / E4B_MXFP4
   int32_t E, N, K, I;       // stack [E, N, K]; I = intermediate size (mode 0 pairing)
   int32_t R;                // routed rows
-  int32_t tokens_per_tile;  // 8 (skinny kernel), 32, 64, 128, 192, 256
+  int32_t tokens_per_tile;  // decode kernel: tokens per chunk (8, 16, 32); tcgen05: tile width (32..256)
+  int32_t decode;           // 1: skinny_gemm (decode kernel), 0: grouped_gemm (tcgen05)
   const uint8_t* codes;     // [E, N, K] packed
   const void* scales;
   const uint16_t* act;      // [R, K] bf16 (x_sorted or h)
@@ -86,8 +88,8 @@ struct GroupedGemmLaunch {
 };
 e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 
-// Decode-sized batches (tokens_per_tile == 8): warp-level MMA with the codes
-// decoded in registers; chunk_off counts chunks of 8 tokens.
+// Decode-sized batches: warp-level MMA with the codes decoded in registers;
+// chunk_off counts chunks of tokens_per_tile (8, 16 or 32) tokens.
 e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 bool skinny_gemm_supported(int32_t K, int32_t fmt);   // the per-unit scale buffers fit in shared memory
 

@@ -68,12 +68,12 @@ constexpr int SK_PRODUCER = 8;                   // warp index
 constexpr int SK_THREADS = 9 * 32;
 constexpr int SK_TPW = 4;                        // MMA tiles per consumer warp
 constexpr int SK_SBUF = 2;                       // per-unit scale buffers
-constexpr int SK_TOK = 8;                        // tokens per chunk (MMA N)
 constexpr int SK_ROWS = 128;                     // weight rows per unit
 constexpr int SK_KST = 256;                      // K per stage
 constexpr int SK_CODE_BYTES = SK_ROWS * SK_KST / 2;          // 16 KB
-constexpr int SK_X_BYTES = SK_TOK * SK_KST * 2;              // 4 KB
-constexpr int SK_STAGE_BYTES = SK_CODE_BYTES + SK_X_BYTES;   // 20 KB
+// a chunk is TG token groups of 8 (MMA N = 8): its activation rows take
+// 4 KB per group and stage; every decoded A fragment feeds TG MMAs
+__host__ __device__ constexpr int sk_stage_bytes(int tg) { return SK_CODE_BYTES + tg * 8 * SK_KST * 2; }
 constexpr int SK_MAX_STAGES = 8;
 // byte table: entry b holds one copy per lane at 256*b + 4*lane (the upper
 // 128 bytes of each entry are unused), so a single byte permute of the code
@@ -109,11 +109,11 @@ struct SkLayout {
   int lut, ring, scale, red, tab, bar, total;
 };
 
-__host__ __device__ inline SkLayout sk_layout(int stages, int scale_bytes) {
+__host__ __device__ inline SkLayout sk_layout(int stages, int scale_bytes, int tg) {
   SkLayout L;
   L.lut = 0;
   L.ring = SK_LUT_BYTES;                                     // 1024-aligned (swizzle atoms)
-  L.scale = L.ring + stages * SK_STAGE_BYTES;
+  L.scale = L.ring + stages * sk_stage_bytes(tg);
   L.red = L.scale + SK_SBUF * scale_bytes;
   L.tab = L.red + SK_RED_BYTES;
   L.bar = L.tab + SK_TAB_BYTES;
@@ -199,6 +199,7 @@ struct Unit {
 
 // Unit u -> (expert, first token, tokens, weight block), from the CTA's copies
 // of chunk_off[E+1] and expert_offsets[E+1].
+template <int TOK>
 __device__ __forceinline__ Unit decode_unit(int u, int n_blocks, int E, const int32_t* s_chunk,
                                             const int32_t* s_off) {
   const int chunk = u / n_blocks;
@@ -210,9 +211,9 @@ __device__ __forceinline__ Unit decode_unit(int u, int n_blocks, int E, const in
     if (s_chunk[mid] <= chunk) lo = mid; else hi = mid;
   }
   r.e = lo;
-  r.t0 = s_off[lo] + SK_TOK * (chunk - s_chunk[lo]);
+  r.t0 = s_off[lo] + TOK * (chunk - s_chunk[lo]);
   const int rem = s_off[lo + 1] - r.t0;
-  r.m = rem < SK_TOK ? rem : SK_TOK;
+  r.m = rem < TOK ? rem : TOK;
   return r;
 }
 
@@ -229,7 +230,7 @@ __device__ __forceinline__ uint32_t lora_pair(const uint16_t* col, int64_t rstri
   return lo | (hi << 16);
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int TG>
 __global__ void __launch_bounds__(SK_THREADS, 1)
     skinny_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ SkParams p) {
@@ -237,7 +238,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   // 1024-aligned base (swizzle atoms), kept as an offset from the shared array so
   // that every access below compiles to a shared-memory load
   uint8_t* smem = sk_dyn + ((1024u - (smem_u32(sk_dyn) & 1023u)) & 1023u);
-  const SkLayout L = sk_layout(p.stages, p.scale_bytes);
+  constexpr int TOK = 8 * TG;                         // tokens per chunk
+  constexpr int STAGE_BYTES = sk_stage_bytes(TG);
+  const SkLayout L = sk_layout(p.stages, p.scale_bytes, TG);
   uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
   const uint8_t* lut_b = smem + L.lut;
   uint8_t* ring = smem + L.ring;
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           mbar_arrive(&sfull[sb]);
           return true;
         }
-        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+        const Unit un = decode_unit<TOK>(u, p.n_blocks, p.E, s_chunk, s_off);
         int row_a, row_b;
         unit_rows<MODE>(p, un, row_a, row_b);
         const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
@@ -351,19 +354,19 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       int u = q0;
       ok = issue_scales(0, u);
       for (int k = 0; ok && u < total; ++k) {
-        const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+        const Unit un = decode_unit<TOK>(u, p.n_blocks, p.E, s_chunk, s_off);
         int row_a, row_b;
         unit_rows<MODE>(p, un, row_a, row_b);
         const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
         for (int st = 0; st < nst; ++st) {
           if (!mbar_wait(&empty[slot], ph ^ 1u, wctx, 712)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[slot], SK_STAGE_BYTES);
-          uint8_t* dst = ring + slot * SK_STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[slot], STAGE_BYTES);
+          uint8_t* dst = ring + slot * STAGE_BYTES;
           tma_load_2d(dst, &tm_codes, &full[slot], SK_KST / 2 * st, ya);
           tma_load_2d(dst + SK_CODE_BYTES / 2, &tm_codes, &full[slot], SK_KST / 2 * st, yb);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            tma_load_2d(dst + SK_CODE_BYTES + 1024 * i, &tm_x, &full[slot], SK_KST * st + 64 * i, un.t0);
+            tma_load_2d(dst + SK_CODE_BYTES + 1024 * TG * i, &tm_x, &full[slot], SK_KST * st + 64 * i, un.t0);
           armed |= 1u << slot;
           par = (par & ~(1u << slot)) | (ph << slot);
           if (++slot == p.stages) { slot = 0; ph ^= 1u; }
@@ -410,8 +413,9 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         so[j][rr] = r[rr] * p.srow;
       }
     }
-    const int xo0 = SK_CODE_BYTES + 1024 * wk + 128 * g + 16 * ((2 * c) ^ g);
-    const int xo1 = SK_CODE_BYTES + 1024 * wk + 128 * g + 16 * ((2 * c + 1) ^ g);
+    // activation box wk holds the chunk's TOK rows x 64 K; row 8tg+g of it feeds token group tg
+    const int xo0 = SK_CODE_BYTES + 1024 * TG * wk + 128 * g + 16 * ((2 * c) ^ g);
+    const int xo1 = SK_CODE_BYTES + 1024 * TG * wk + 128 * g + 16 * ((2 * c + 1) ^ g);
     // the scale buffer's swizzle flips bits 4..6 by bits 7..9 of the row offset,
     // which are the same for every row this lane reads
     const uint32_t xg = (static_cast<uint32_t>(so[0][0]) >> 3) & p.scale_swz;
@@ -422,20 +426,27 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       if (!warp_wait(&sfull[sb], sph, wctx, 721)) break;
       const int u = s_unit[sb];
       if (u < 0) break;
-      const Unit un = decode_unit(u, p.n_blocks, p.E, s_chunk, s_off);
+      const Unit un = decode_unit<TOK>(u, p.n_blocks, p.E, s_chunk, s_off);
       const uint8_t* scb = sbuf + sb * p.scale_bytes;
-      float acc[SK_TPW][4];
+      float acc[SK_TPW][TG][4];
 #pragma unroll
-      for (int j = 0; j < SK_TPW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int j = 0; j < SK_TPW; ++j)
+#pragma unroll
+        for (int q = 0; q < TG; ++q) acc[j][q][0] = acc[j][q][1] = acc[j][q][2] = acc[j][q][3] = 0.f;
       for (int st = 0; st < nst; ++st) {
         if (!warp_wait(&full[slot], ph, wctx, 722)) { ok = false; break; }
         const int blk = 4 * st + wk;
         if (blk < KB) {
-          const uint8_t* cs = ring + slot * SK_STAGE_BYTES;
+          const uint8_t* cs = ring + slot * STAGE_BYTES;
           const uint8_t* sc = scb + ((static_cast<uint32_t>(blk * esz)) ^ xg);
-          const uint4 xa = *reinterpret_cast<const uint4*>(cs + xo0);
-          const uint4 xb = *reinterpret_cast<const uint4*>(cs + xo1);
-          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          uint32_t xw[TG][8];
+#pragma unroll
+          for (int q = 0; q < TG; ++q) {
+            const uint4 xa = *reinterpret_cast<const uint4*>(cs + xo0 + 1024 * q);
+            const uint4 xb = *reinterpret_cast<const uint4*>(cs + xo1 + 1024 * q);
+            xw[q][0] = xa.x; xw[q][1] = xa.y; xw[q][2] = xa.z; xw[q][3] = xa.w;
+            xw[q][4] = xb.x; xw[q][5] = xb.y; xw[q][6] = xb.z; xw[q][7] = xb.w;
+          }
 #pragma unroll
           for (int j = 0; j < SK_TPW; ++j) {
             const uint2 q0 = *reinterpret_cast<const uint2*>(cs + co[j][0]);
@@ -445,21 +456,27 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             const uint32_t s1 = FMT == E4B_NF4 ? *reinterpret_cast<const uint32_t*>(sc + so[j][1])
                                                : *reinterpret_cast<const uint16_t*>(sc + so[j][1]);
             if (FMT == E4B_NF4) {
-              float bs[4];
+              float bs[TG][4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const uint32_t w0 = i < 2 ? q0.x : q0.y, w1 = i < 2 ? q1.x : q1.y;
                 const int by = 2 * (i & 1);
                 const uint32_t a[4] = {lut_at(lut_b, lane_off, w0, by), lut_at(lut_b, lane_off, w1, by),
                                        lut_at(lut_b, lane_off, w0, by + 1), lut_at(lut_b, lane_off, w1, by + 1)};
-                if (i == 0) mma_bf16_z(bs, a, xw[0], xw[1]);
-                else mma_bf16(bs, a, xw[2 * i], xw[2 * i + 1]);
+#pragma unroll
+                for (int q = 0; q < TG; ++q) {
+                  if (i == 0) mma_bf16_z(bs[q], a, xw[q][0], xw[q][1]);
+                  else mma_bf16(bs[q], a, xw[q][2 * i], xw[q][2 * i + 1]);
+                }
               }
               const float f0 = __uint_as_float(s0), f1 = __uint_as_float(s1);
-              acc[j][0] = fmaf(f0, bs[0], acc[j][0]);
-              acc[j][1] = fmaf(f0, bs[1], acc[j][1]);
-              acc[j][2] = fmaf(f1, bs[2], acc[j][2]);
-              acc[j][3] = fmaf(f1, bs[3], acc[j][3]);
+#pragma unroll
+              for (int q = 0; q < TG; ++q) {
+                acc[j][q][0] = fmaf(f0, bs[q][0], acc[j][q][0]);
+                acc[j][q][1] = fmaf(f0, bs[q][1], acc[j][q][1]);
+                acc[j][q][2] = fmaf(f1, bs[q][2], acc[j][q][2]);
+                acc[j][q][3] = fmaf(f1, bs[q][3], acc[j][q][3]);
+              }
             } else {
               const uint32_t e0 = e8m0_bf16x2((s0 >> (8 * (c >> 1))) & 0xFFu);
               const uint32_t e1 = e8m0_bf16x2((s1 >> (8 * (c >> 1))) & 0xFFu);
@@ -471,7 +488,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
                                        bf16x2_mul(lut_at(lut_b, lane_off, w1, by), e1),
                                        bf16x2_mul(lut_at(lut_b, lane_off, w0, by + 1), e0),
                                        bf16x2_mul(lut_at(lut_b, lane_off, w1, by + 1), e1)};
-                mma_bf16(acc[j], a, xw[2 * i], xw[2 * i + 1]);
+#pragma unroll
+                for (int q = 0; q < TG; ++q) mma_bf16(acc[j][q], a, xw[q][2 * i], xw[q][2 * i + 1]);
               }
             }
           }
@@ -483,77 +501,86 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sempty[sb]);
-      // sum the four K-partials of each tile; warp (wr, wk < SK_TPW) finishes tile SK_TPW*wr+wk
-      if (!warp_wait(rempty, rph ^ 1u, wctx, 723)) break;
-#pragma unroll
-      for (int j = 0; j < SK_TPW; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) red[((warp * SK_TPW + j) * 4 + i) * 32 + lane] = acc[j][i];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(rfull);
-      if (wk >= SK_TPW) {
-        rph ^= 1u;
-        if (++sb == SK_SBUF) { sb = 0; sph ^= 1u; }
-        continue;
-      }
-      if (!warp_wait(rfull, rph, wctx, 724)) break;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] += red[(((4 * wr + k) * SK_TPW + wk) * 4 + i) * 32 + lane];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(rempty);
-      rph ^= 1u;
+      // sum the four K-partials of each tile, one token group per round; warp
+      // (wr, wk < SK_TPW) finishes tile SK_TPW*wr+wk
       const int t = SK_TPW * wr + wk;
-      if (MODE == 0) {
+      const bool fin = wk < SK_TPW;
+      uint32_t la[4] = {0u, 0u, 0u, 0u};             // LoRA step A fragment of the finished tile
+      if (MODE == 0 && fin && p.lora_rank > 0) {
         const int col = 64 * un.nb + 8 * t + rho;
-        if (p.lora_rank > 0) {
-          // LoRA step: A = B_e^T (rows n, K = rank padded to 16), B = xa (scale folded in)
-          uint32_t b0 = 0u, b1 = 0u;
-          if (g < un.m) {
-            const uint32_t* xr = reinterpret_cast<const uint32_t*>(p.xa + static_cast<int64_t>(un.t0 + g) * 64);
-            b0 = __ldg(xr + c);
-            b1 = __ldg(xr + 4 + c);
-          }
-          const int64_t rs = 2 * static_cast<int64_t>(p.I);
-          const uint16_t* Be = p.lora_B + static_cast<int64_t>(un.e) * p.lora_rank * rs;
-          const uint32_t a[4] = {lora_pair(Be + col, rs, 2 * c, p.lora_rank),
-                                 lora_pair(Be + p.I + col, rs, 2 * c, p.lora_rank),
-                                 lora_pair(Be + col, rs, 2 * c + 8, p.lora_rank),
-                                 lora_pair(Be + p.I + col, rs, 2 * c + 8, p.lora_rank)};
-          mma_bf16(v, a, b0, b1);
-        }
-        __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (2 * c + q < un.m) {
-            const float gt = v[q], up = v[2 + q];
-            const float sg = __fdividef(gt, 1.0f + __expf(-gt));
-            h[static_cast<int64_t>(un.t0 + 2 * c + q) * p.I + col] = __float2bfloat16_rn(sg * up);
-          }
-        }
-      } else {
-        const int n = SK_ROWS * un.nb + 16 * t + rho;
-        float* y = static_cast<float*>(p.out);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          if (2 * c + q < un.m) {
-            float* yr = y + static_cast<int64_t>(un.t0 + 2 * c + q) * p.N + n;
-            if (n < p.N) yr[0] = v[q];
-            if (n + 8 < p.N) yr[8] = v[2 + q];
-          }
-        }
+        const int64_t rs = 2 * static_cast<int64_t>(p.I);
+        const uint16_t* Be = p.lora_B + static_cast<int64_t>(un.e) * p.lora_rank * rs;
+        la[0] = lora_pair(Be + col, rs, 2 * c, p.lora_rank);
+        la[1] = lora_pair(Be + p.I + col, rs, 2 * c, p.lora_rank);
+        la[2] = lora_pair(Be + col, rs, 2 * c + 8, p.lora_rank);
+        la[3] = lora_pair(Be + p.I + col, rs, 2 * c + 8, p.lora_rank);
       }
+#pragma unroll
+      for (int q = 0; q < TG; ++q) {
+        if (!warp_wait(rempty, rph ^ 1u, wctx, 723)) { ok = false; break; }
+#pragma unroll
+        for (int j = 0; j < SK_TPW; ++j)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) red[((warp * SK_TPW + j) * 4 + i) * 32 + lane] = acc[j][q][i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(rfull);
+        if (fin) {
+          if (!warp_wait(rfull, rph, wctx, 724)) { ok = false; break; }
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] += red[(((4 * wr + k) * SK_TPW + wk) * 4 + i) * 32 + lane];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(rempty);
+          const int tok0 = 8 * q;                    // first token of this group in the chunk
+          if (MODE == 0) {
+            const int col = 64 * un.nb + 8 * t + rho;
+            if (p.lora_rank > 0) {
+              // LoRA step: A = B_e^T (rows n, K = rank padded to 16), B = xa (scale folded in)
+              uint32_t b0 = 0u, b1 = 0u;
+              if (tok0 + g < un.m) {
+                const uint32_t* xr =
+                    reinterpret_cast<const uint32_t*>(p.xa + static_cast<int64_t>(un.t0 + tok0 + g) * 64);
+                b0 = __ldg(xr + c);
+                b1 = __ldg(xr + 4 + c);
+              }
+              mma_bf16(v, la, b0, b1);
+            }
+            __nv_bfloat16* h = static_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              if (tok0 + 2 * c + r < un.m) {
+                const float gt = v[r], up = v[2 + r];
+                const float sg = __fdividef(gt, 1.0f + __expf(-gt));
+                h[static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.I + col] = __float2bfloat16_rn(sg * up);
+              }
+            }
+          } else {
+            const int n = SK_ROWS * un.nb + 16 * t + rho;
+            float* y = static_cast<float*>(p.out);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              if (tok0 + 2 * c + r < un.m) {
+                float* yr = y + static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.N + n;
+                if (n < p.N) yr[0] = v[r];
+                if (n + 8 < p.N) yr[8] = v[2 + r];
+              }
+            }
+          }
+        }
+        rph ^= 1u;
+      }
+      if (!ok) break;
       if (++sb == SK_SBUF) { sb = 0; sph ^= 1u; }
     }
   }
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int TG>
 e4b_status launch_typed(const CUtensorMap& tc, const CUtensorMap& tx, const CUtensorMap& ts, const SkParams& prm,
                         int smem, cudaStream_t s) {
-  auto kern = skinny_gemm_kernel<FMT, MODE>;
+  auto kern = skinny_gemm_kernel<FMT, MODE, TG>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -570,13 +597,26 @@ int scale_buffer_bytes(int32_t K, int32_t fmt) { return (SK_ROWS * scale_row_byt
 }  // namespace
 
 bool skinny_gemm_supported(int32_t K, int32_t fmt) {
-  return sk_layout(3, scale_buffer_bytes(K, fmt)).total <= SK_SMEM_LIMIT;
+  return sk_layout(3, scale_buffer_bytes(K, fmt), 4).total <= SK_SMEM_LIMIT;
+}
+
+template <int TG>
+e4b_status launch_tg(int32_t fmt, int32_t mode, const CUtensorMap& tc, const CUtensorMap& tx, const CUtensorMap& ts,
+                     const SkParams& prm, int smem, cudaStream_t s) {
+  if (fmt == E4B_NF4)
+    return mode == 0 ? launch_typed<E4B_NF4, 0, TG>(tc, tx, ts, prm, smem, s)
+                     : launch_typed<E4B_NF4, 1, TG>(tc, tx, ts, prm, smem, s);
+  return mode == 0 ? launch_typed<E4B_MXFP4, 0, TG>(tc, tx, ts, prm, smem, s)
+                   : launch_typed<E4B_MXFP4, 1, TG>(tc, tx, ts, prm, smem, s);
 }
 
 e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   if (g.R == 0) return E4B_OK;
-  if (g.K % 64 != 0 || (g.mode == 0 && g.I % 64 != 0) || !skinny_gemm_supported(g.K, g.fmt))
+  const int tok = g.tokens_per_tile;                  // 8, 16 or 32 tokens per chunk
+  if (g.K % 64 != 0 || (g.mode == 0 && g.I % 64 != 0) || !skinny_gemm_supported(g.K, g.fmt) ||
+      (tok != 8 && tok != 16 && tok != 32))
     return E4B_ERR_UNSUPPORTED;
+  const int tg = tok / 8;
   SkParams prm;
   prm.E = g.E;
   prm.N = g.N;
@@ -591,7 +631,7 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.scale_tma = (prm.srow == 32 || prm.srow == 64 || prm.srow == 128) ? 1 : 0;
   prm.scale_swz = prm.scale_tma ? static_cast<uint32_t>(((prm.srow >> 4) - 1) << 4) : 0u;
   int stages = SK_MAX_STAGES;
-  while (stages > 3 && sk_layout(stages, prm.scale_bytes).total > SK_SMEM_LIMIT) --stages;
+  while (stages > 3 && sk_layout(stages, prm.scale_bytes, tg).total > SK_SMEM_LIMIT) --stages;
   prm.stages = stages;
   prm.codes = g.codes;
   prm.scales = g.scales;
@@ -616,7 +656,7 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return E4B_ERR_CUDA;
   if (!encode_tma_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, 64,
-                     SK_TOK, CU_TENSOR_MAP_SWIZZLE_128B))
+                     tok, CU_TENSOR_MAP_SWIZZLE_128B))
     return E4B_ERR_CUDA;
   if (prm.scale_tma) {
     const CUtensorMapSwizzle sw = prm.srow == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -627,12 +667,10 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   } else {
     ts = tc;
   }
-  const int smem = sk_layout(stages, prm.scale_bytes).total;
-  if (g.fmt == E4B_NF4)
-    return g.mode == 0 ? launch_typed<E4B_NF4, 0>(tc, tx, ts, prm, smem, s)
-                       : launch_typed<E4B_NF4, 1>(tc, tx, ts, prm, smem, s);
-  return g.mode == 0 ? launch_typed<E4B_MXFP4, 0>(tc, tx, ts, prm, smem, s)
-                     : launch_typed<E4B_MXFP4, 1>(tc, tx, ts, prm, smem, s);
+  const int smem = sk_layout(stages, prm.scale_bytes, tg).total;
+  if (tg == 1) return launch_tg<1>(g.fmt, g.mode, tc, tx, ts, prm, smem, s);
+  if (tg == 2) return launch_tg<2>(g.fmt, g.mode, tc, tx, ts, prm, smem, s);
+  return launch_tg<4>(g.fmt, g.mode, tc, tx, ts, prm, smem, s);
 }
 
 }  // namespace e4b

@@ -85,9 +85,10 @@ typedef struct {
   int32_t act;             /* E4B_ACT_SWIGLU */
   int32_t tokens_per_tile; /* 0 = chosen by the library (the decode kernel when the mean number of rows
                               per routed expert is at most 12, else a tcgen05 tile); 8 = decode kernel
-                              (codes decoded in registers, warp-level MMA, chunks of 8 tokens; needs the
-                              scale rows of 128 weight rows of both stacks to fit in shared memory, else
-                              E4B_ERR_UNSUPPORTED); 32, 64, 128, 192 or 256 = tcgen05 tile width */
+                              (codes decoded in registers, warp-level MMA; tokens go in chunks of 8, 16
+                              or 32 by the mean rows per expert; needs the scale rows of 128 weight rows
+                              of both stacks to fit in shared memory, else E4B_ERR_UNSUPPORTED);
+                              32, 64, 128, 192 or 256 = tcgen05 tile width */
 } e4b_moe_desc;
 
 /* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */
