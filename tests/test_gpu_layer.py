@@ -58,6 +58,15 @@ def test_k_equals_e_and_one_expert_takes_all(tpt):
     run_and_compare(w1, 700, tokens_per_tile=tpt, x=x, logits=synth.to_bf16_bits(lg))
 
 
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+@pytest.mark.parametrize("T", [30, 100, 180])
+def test_decode_kernel_chunk_sizes(fmt, T):
+    # E=16, k=2: mean rows per expert 3.75 / 12.5 / 22.5 -> chunks of 8 / 16 / 32 tokens, with
+    # experts whose counts straddle chunk boundaries; K = 320 and 192 leave ragged last stages
+    w = Workload(f"chunks_{fmt}", fmt, E=16, H=320, I=192, k=2, tokens=(T,), exp_range=(-4, 2), seed=11)
+    run_and_compare(w, T, tokens_per_tile=8)
+
+
 @pytest.mark.parametrize("tpt", [0, 8])
 @pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
 def test_lora_tiny_and_zero_b(fmt, tpt):
