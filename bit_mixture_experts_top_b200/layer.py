@@ -70,6 +70,51 @@ class MoeLayer:
         return self._ws[off:off + nbytes].view(dtype)
 
 
+class HostForward:
+    """Host-to-host forward at a fixed batch size, for serving loops.
+
+    The caller writes bf16 bit patterns into the pinned staging tensors ``x`` [T, H] and
+    ``logits`` [T, E]; :meth:`run` copies them to the device, runs the layer and copies the
+    result into the pinned ``out`` [T, H], all replayed from one CUDA graph captured on the
+    first call (the graph holds the copies and the library's launches, so a step costs one
+    graph launch instead of one launch per kernel).  The layer's workspace and the device
+    buffers are owned by this object and must not be resized while it is in use."""
+
+    def __init__(self, layer: "MoeLayer", T: int, device):
+        self.layer, self.T, self.device = layer, T, torch.device(device)
+        self.x = torch.empty((T, layer.H), dtype=torch.int16).pin_memory()
+        self.logits = torch.empty((T, layer.E), dtype=torch.int16).pin_memory()
+        self.out = torch.empty((T, layer.H), dtype=torch.int16).pin_memory()
+        self._x = torch.empty((T, layer.H), dtype=torch.int16, device=self.device)
+        self._lg = torch.empty((T, layer.E), dtype=torch.int16, device=self.device)
+        self._out = torch.empty((T, layer.H), dtype=torch.int16, device=self.device)
+        layer.workspace(T, self.device)
+        self._graph = None
+
+    def _step(self):
+        self._x.copy_(self.x, non_blocking=True)
+        self._lg.copy_(self.logits, non_blocking=True)
+        self.layer.forward(self._x, self._lg, out=self._out)
+        self.out.copy_(self._out, non_blocking=True)
+
+    def run(self):
+        """One forward from ``x``/``logits`` to ``out``; returns ``out`` after the device finished."""
+        if self._graph is None:
+            side = torch.cuda.Stream(device=self.device)
+            side.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(side):          # first call outside capture: one-time set-up
+                self._step()
+            torch.cuda.current_stream(self.device).wait_stream(side)
+            torch.cuda.synchronize(self.device)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._step()
+            self._graph = g
+        self._graph.replay()
+        torch.cuda.current_stream(self.device).synchronize()
+        return self.out
+
+
 def bits_tensor(bits_np, device):
     """uint16 bf16 bit patterns (NumPy) -> a bf16 device tensor."""
     return torch.from_numpy(np.ascontiguousarray(bits_np).view(np.int16)).to(device).view(torch.bfloat16)

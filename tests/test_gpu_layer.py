@@ -146,3 +146,20 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert e4b.e4b_device_status(ws) == e4b.E4B_ERR_TIMEOUT
     assert e4b.e4b_device_status(ws) == e4b.E4B_OK          # cleared by the read
     run_and_compare(TINY, 64)                               # the context still works
+
+
+def test_host_forward_graph_replay_matches_forward():
+    # the graph-replayed host-to-host call gives the stream call's bits, and picks up
+    # new inputs written into its staging tensors between replays
+    dev = device()
+    lay = layer.synthetic_layer(QWEN, dev)
+    hf = layer.HostForward(lay, 64, dev)
+    for seed_offset in (0, 1):
+        x, lg = layer.synthetic_tokens(QWEN, 64, seed_offset)
+        hf.x.copy_(torch.from_numpy(x.view(np.int16)))
+        hf.logits.copy_(torch.from_numpy(lg.view(np.int16)))
+        got = hf.run().clone()
+        ref = lay.forward(layer.bits_tensor(x, dev), layer.bits_tensor(lg, dev))
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref.view(torch.int16).cpu())
+    assert e4b.e4b_device_status(lay._ws) == e4b.E4B_OK
