@@ -327,7 +327,45 @@ def bench_e4b(args, world, rank, local):
     d2h_bytes = int(hf.out.numel() * 2)
     del hf
 
+    # the two standalone format kernels on their full stacks (inputs larger than L2, timed per launch)
+    formats = {}
+    if args.workload == WORKLOAD and not args.no_formats:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(0)
+        n_q = 128 * 2048 * 1536                      # the Qwen3-shaped gate_up stack, fp32 N(0, 0.02)
+        xq = torch.empty(n_q, dtype=torch.float32, device=dev).normal_(0.0, 0.02, generator=gen)
+        cq = torch.empty(n_q // 2, dtype=torch.uint8, device=dev)
+        aq = torch.empty(n_q // 64, dtype=torch.float32, device=dev)
+        n_d = 32 * 2880 * 5760                       # the gpt-oss-20b-shaped gate_up stack
+        cd = torch.randint(0, 256, (n_d // 2,), dtype=torch.uint8, device=dev, generator=gen)
+        sd = torch.randint(121, 129, (n_d // 32,), dtype=torch.uint8, device=dev, generator=gen)
+        od = torch.empty(n_d, dtype=torch.int16, device=dev)
+
+        def time_calls(fn, n=20):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            evs[0].record()
+            for i in range(n):
+                fn()
+                evs[i + 1].record()
+            torch.cuda.synchronize()
+            return statistics.fmean(evs[i].elapsed_time(evs[i + 1]) for i in range(n))
+
+        q_ms = max_over_ranks(time_calls(lambda: e4b.e4b_quantize_nf4(xq, n_q, cq, aq)))
+        d_ms = max_over_ranks(time_calls(lambda: e4b.e4b_dequant_mxfp4(cd, sd, n_d, od)))
+        q_bytes = n_q * 4 + n_q // 2 + n_q // 64 * 4
+        d_bytes = n_d // 2 + n_d // 32 + n_d * 2
+        formats = {"quantize_nf4": {"shape": [128, 2048, 1536], "ms": q_ms, "bytes": q_bytes,
+                                    "gbs": q_bytes / (q_ms * 1e-3) / 1e9},
+                   "dequant_mxfp4": {"shape": [32, 2880, 5760], "ms": d_ms, "bytes": d_bytes,
+                                     "gbs": d_bytes / (d_ms * 1e-3) / 1e9}}
+        del xq, cq, aq, cd, sd, od
+
     peaks, peak_kind = load_peaks()
+    for f in formats.values():
+        f["frac_of_hbm"] = f["gbs"] / peaks["hbm_gbs"]
     # the library's kernel choice (tokens_per_tile 0): the decode kernel at <= 12 rows per routed expert
     active = min(R, w.E)
     decode_kernel = (R + active - 1) // active <= 12
@@ -364,6 +402,7 @@ def bench_e4b(args, world, rank, local):
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "path": "layer.HostForward.run: pinned host inputs -> device -> forward -> pinned host output, "
                         "one CUDA graph replay and a synchronize per step"},
+        "standalone_kernels": formats,
         "gpu_launches": K * KERNELS_PER_STEP,
         "clocks": clocks,
     }
@@ -389,6 +428,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--no-formats", action="store_true", help="skip timing the standalone format kernels")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD,
                     help="synthetic layer to time (default: the headline decode workload)")
     ap.add_argument("--tokens", type=int, default=None, help="tokens per step (default: the workload's largest)")

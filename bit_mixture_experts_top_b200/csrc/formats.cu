@@ -36,28 +36,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 8 elements = 4 code bytes -> 16 output bytes.  Unit u covers elements [8u, 8u+8).
+__device__ __forceinline__ uint4 decode_unit8(uint32_t w, uint32_t s) {
+  if (s == 255u) return make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+  const float sc = e8m0_to_f32(s);
+  uint32_t r[4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t byte = (w >> (8 * b)) & 0xFFu;
+    r[b] = pack_bf16x2(e2m1_to_f32(byte & 0xFu) * sc, e2m1_to_f32(byte >> 4) * sc);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+// 8 elements = 4 code bytes -> 16 output bytes.  Unit u covers elements [8u, 8u+8);
+// each thread takes two units per trip (u and u + stride) so two loads are in flight.
 __global__ void __launch_bounds__(256) dequant_mxfp4_kernel(const uint32_t* __restrict__ codes,
                                                               const uint8_t* __restrict__ scales, int64_t units,
                                                               uint4* __restrict__ out) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units; u += stride) {
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units; u += 2 * stride) {
+    const int64_t u2 = u + stride;
+    const bool two = u2 < units;
     const uint32_t w = __ldcs(codes + u);
     const uint32_t s = __ldg(scales + (u >> 2));
-    uint4 o;
-    if (s == 255u) {
-      o = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
-    } else {
-      const float sc = e8m0_to_f32(s);
-      uint32_t r[4];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t byte = (w >> (8 * b)) & 0xFFu;
-        r[b] = pack_bf16x2(e2m1_to_f32(byte & 0xFu) * sc, e2m1_to_f32(byte >> 4) * sc);
-      }
-      o = make_uint4(r[0], r[1], r[2], r[3]);
-    }
-    __stcs(out + u, o);
+    const uint32_t w2 = two ? __ldcs(codes + u2) : 0u;
+    const uint32_t s2 = two ? __ldg(scales + (u2 >> 2)) : 0u;
+    __stcs(out + u, decode_unit8(w, s));
+    if (two) __stcs(out + u2, decode_unit8(w2, s2));
   }
 }
 
@@ -65,8 +70,44 @@ struct Nf4Mids {
   float m[15];
 };
 
-// One half-warp per 64-block: each lane loads 4 consecutive fp32 (16 bytes),
+// One half-warp per 64-block: each lane holds 4 consecutive fp32 (16 bytes),
 // the half-warp reduces |x| to absmax, each lane emits 4 codes (2 bytes).
+__device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_t half_mask, float m7,
+                                              const float* s_mid, uint16_t* __restrict__ codes,
+                                              float* __restrict__ absmax) {
+  float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
+  uint32_t c[4];
+  const float xv[4] = {v.x, v.y, v.z, v.w};
+  // y = fl32(x / a) by Markstein's FMA correction (P. Markstein, "Computation of
+  // elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev.
+  // 34(1), 1990): with r = RN(1/a), q = RN(x*r), the residual x - a*q is exact in
+  // one FMA and RN(q + residual*r) is the correctly rounded quotient unless it
+  // underflows.  |x| <= a here, and an underflowing quotient lies far below the
+  // smallest decision midpoint, so the code is the same either way.
+  const float r = __frcp_rn(a);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (a == 0.0f) {
+      c[i] = 7u;
+    } else {
+      const float q = xv[i] * r;
+      const float y = fmaf(fmaf(-a, q, xv[i]), r, q);
+      uint32_t k = (y > m7) ? 8u : 0u;        // count of midpoints below y, by bisection
+      k += (y > s_mid[k + 3]) ? 4u : 0u;
+      k += (y > s_mid[k + 1]) ? 2u : 0u;
+      k += (y > s_mid[k]) ? 1u : 0u;
+      c[i] = k;
+    }
+  }
+  const uint32_t b0 = (c[0] << 4) | c[1];
+  const uint32_t b1 = (c[2] << 4) | c[3];
+  codes[q] = static_cast<uint16_t>(b0 | (b1 << 8));
+  if ((threadIdx.x & 15) == 0) absmax[q >> 4] = a;
+}
+
+// Each thread takes two quads per trip (q and q + stride): two loads in flight.
 __global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restrict__ x, int64_t quads,
                                                              uint16_t* __restrict__ codes,
                                                              float* __restrict__ absmax, Nf4Mids mids) {
@@ -75,33 +116,15 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restr
   __syncthreads();
   const float m7 = mids.m[7];
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  // quads is a multiple of 16, so every half-warp stays inside one block and
-  // the loop trip count is uniform across each half-warp.
-  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < quads; q += stride) {
+  const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16u);   // this half-warp only
+  // quads and the stride are multiples of 16, so every half-warp stays inside one
+  // block and the trip count and the second-quad test are uniform across it.
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < quads; q += 2 * stride) {
+    const int64_t q2 = q + stride;
     const float4 v = __ldcs(x + q);
-    float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16u);   // this half-warp only
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
-    uint32_t c[4];
-    const float xv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (a == 0.0f) {
-        c[i] = 7u;
-      } else {
-        const float y = __fdiv_rn(xv[i], a);
-        uint32_t k = (y > m7) ? 8u : 0u;        // count of midpoints below y, by bisection
-        k += (y > s_mid[k + 3]) ? 4u : 0u;
-        k += (y > s_mid[k + 1]) ? 2u : 0u;
-        k += (y > s_mid[k]) ? 1u : 0u;
-        c[i] = k;
-      }
-    }
-    const uint32_t b0 = (c[0] << 4) | c[1];
-    const uint32_t b1 = (c[2] << 4) | c[3];
-    codes[q] = static_cast<uint16_t>(b0 | (b1 << 8));
-    if ((threadIdx.x & 15) == 0) absmax[q >> 4] = a;
+    const float4 v2 = q2 < quads ? __ldcs(x + q2) : make_float4(0.f, 0.f, 0.f, 0.f);
+    quantize_quad(v, q, half_mask, m7, s_mid, codes, absmax);
+    if (q2 < quads) quantize_quad(v2, q2, half_mask, m7, s_mid, codes, absmax);
   }
 }
 

@@ -94,6 +94,31 @@ def test_quantize_nf4_codebook_roundtrip_and_midpoints():
     assert np.array_equal(onf4.unpack_nf4(codes, 64), np.tile(np.arange(16, dtype=np.uint8), 4))
 
 
+def test_quantize_nf4_quotients_next_to_midpoints():
+    # x / a lands within a few ulps of a decision midpoint for arbitrary (non power of
+    # two) absmax a: the cases where the rounding of the quotient decides the code
+    g = np.random.default_rng(21)
+    mids = onf4.nf4_midpoints()
+    blocks = []
+    for _ in range(4000):
+        a = np.float32(g.uniform(0.5, 2.0) * 2.0 ** g.integers(-20, 20))
+        b = np.empty(64, np.float32)
+        b[0] = a                                                 # the block's absmax
+        i = g.integers(0, 15, 63)
+        base = (mids[i].astype(np.float64) * np.float64(a)).astype(np.float32)
+        steps = g.integers(-3, 4, 63)
+        b[1:] = [np.float32(v) for v in base]
+        for j, st in enumerate(steps):
+            v = b[1 + j]
+            for _ in range(abs(int(st))):
+                v = np.nextafter(v, np.float32(np.inf) if st > 0 else np.float32(-np.inf))
+            b[1 + j] = v
+        b[1:] *= np.where(g.random(63) < 0.5, -1, 1).astype(np.float32)
+        b[1:] = np.clip(b[1:], -a, a)
+        blocks.append(b)
+    _assert_quant_equal(np.concatenate(blocks))
+
+
 @pytest.mark.parametrize("n", [64, 128, 192, 64 * 17, 64 * 1000 + 64])
 def test_quantize_nf4_ragged_sizes(n):
     x = (np.random.default_rng(n).standard_normal(n) * 0.02).astype(np.float32)
