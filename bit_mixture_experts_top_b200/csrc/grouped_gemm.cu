@@ -50,14 +50,12 @@ constexpr int RAW_K = 128;                   // K per packed-code stage
 constexpr int RAW_ROW_BYTES = RAW_K / 2;     // 64 bytes of codes per weight row
 constexpr int RAW_STAGE_BYTES = BM * RAW_ROW_BYTES;
 constexpr int LUT_BYTES = 32768;             // byte -> element-pair table, one copy per bank
-constexpr int NUM_DQ_WARPS = 8;
+constexpr int NUM_DQ_WARPS = 8;             // dequant warps that produce one A stage (4 lane quarters x 2)
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int WARP_RAW = 0;                  // TMA producer of packed codes
 constexpr int WARP_ACT = 1;                  // TMA producer of activation tiles
 constexpr int WARP_MMA = 2;
 constexpr int WARP_DQ0 = 3;
-constexpr int WARP_EPI0 = WARP_DQ0 + NUM_DQ_WARPS;
-constexpr int NUM_THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
 
@@ -81,6 +79,11 @@ struct Cfg {
   static constexpr int B_ATOM_BYTES = BN * 128;
   static constexpr int B_STAGE_BYTES = ATOMS * B_ATOM_BYTES;
   static constexpr int RAW_STAGES = BN <= 64 ? 12 : (TMEM_A ? 6 : 4);
+  // 64-K stages (prefill tiles): two groups of 8 dequant warps take alternate
+  // 128-K code stages, so each warp converts and synchronises half as often
+  static constexpr int DQ_GROUPS = BKS == 64 ? 2 : 1;
+  static constexpr int WARP_EPI0 = WARP_DQ0 + NUM_DQ_WARPS * DQ_GROUPS;
+  static constexpr int THREADS = 32 * (WARP_EPI0 + NUM_EPI_WARPS);
   static constexpr int TMEM_COLS = 512;
   static constexpr int OFF_LUT = 0;
   static constexpr int OFF_A = OFF_LUT + LUT_BYTES;
@@ -213,7 +216,7 @@ __device__ __forceinline__ uint64_t dup_f32(float a) {
 }
 
 template <int BN, int FMT, int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_act,
                         const __grid_constant__ CUtensorMap tm_xa, const Params p) {
   using C = Cfg<BN>;
@@ -259,19 +262,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // bf16 pairs (32 copies of 4 bytes).
   if (FMT == E4B_NF4) {
     float2* lut = reinterpret_cast<float2*>(sLut);
-    for (int i = threadIdx.x; i < 256 * 16; i += NUM_THREADS) {
+    for (int i = threadIdx.x; i < 256 * 16; i += C::THREADS) {
       const int b = i >> 4;
       lut[i] = make_float2(p.lut[b >> 4], p.lut[b & 15]);
     }
   } else {
     uint32_t* lut = reinterpret_cast<uint32_t*>(sLut);
-    for (int i = threadIdx.x; i < 256 * 32; i += NUM_THREADS) {
+    for (int i = threadIdx.x; i < 256 * 32; i += C::THREADS) {
       const int b = i >> 5;
       __nv_bfloat162 v = __floats2bfloat162_rn(e2m1_to_f32(b & 15), e2m1_to_f32(b >> 4));
       lut[i] = *reinterpret_cast<uint32_t*>(&v);
     }
   }
-  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
+  for (int i = threadIdx.x; i <= p.E; i += C::THREADS) {
     s_chunk[i] = __ldg(p.chunk_off + i);
     s_off[i] = __ldg(p.expert_offsets + i);
   }
@@ -424,13 +427,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok && issued) mbar_drain(last_bar, last_par, kDrainNs);   // MMAs in flight finish first
     }
-  } else if (warp < WARP_EPI0) {
+  } else if (warp < C::WARP_EPI0) {
     // ------------------------------------------------------------ dequant
     // With A in tensor memory, A row = TMEM lane and a warp may only touch its
     // own quarter of the lanes; with A in shared memory any mapping works.
     const int quarter = warp & 3;
     const int prow = 32 * quarter + lane;          // A-tile row written by this thread
-    const int half = (warp - WARP_DQ0) >> 2;       // BKS 128: atom; BKS 64: 32-element half of the atom
+    const int half = ((warp - WARP_DQ0) >> 2) & 1; // BKS 128: atom; BKS 64: 32-element half of the atom
+    const int group = (warp - WARP_DQ0) >> 3;      // BKS 64: takes the 128-K code stages of its parity
+    int64_t gs = 0, gr = 0;                        // BKS 64: MMA / code stages of the tiles before this one
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(32 * quarter) << 16);
     const uint32_t lut_l =
         smem_u32(sLut) + (FMT == E4B_NF4 ? static_cast<uint32_t>(lane & 15) * 8u : static_cast<uint32_t>(lane) * 4u);
@@ -493,47 +498,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
         }
       } else {
-        // each thread: 32 elements (half of one 64-wide atom row) per MMA stage
-        auto load_scale = [&](int ks, uint64_t& a2, uint32_t& s2) {
-          if (FMT == E4B_NF4) a2 = dup_f32(__ldg(sc_nf4 + ks));
-          else s2 = e8m0_to_bf16x2(__ldg(sc_mx + 2 * ks + half));
-        };
+        // each thread: 32 elements (half of one 64-wide atom row) per MMA stage; the
+        // group takes code stage j of the tile when gr + j has its parity
         const int ksteps = p.K / ATOM_K;
-        uint64_t a2n = 0;
-        uint32_t s2n = 0;
-        load_scale(0, a2n, s2n);
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint64_t a2 = a2n;
-          const uint32_t s2 = s2n;
-          if (ks + 1 < ksteps) load_scale(ks + 1, a2n, s2n);
-          if ((ks & 1) == 0 && !mbar_wait(&raw_full[rstage], rphase, wctx, 301)) { ok = false; break; }
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wctx, 302)) { ok = false; break; }
-          const uint8_t* raw = sRaw + rstage * RAW_STAGE_BYTES;
-          const uint4 q = *reinterpret_cast<const uint4*>(
-              raw + swizzled_offset(raw_row, (ks & 1) * 2 + half, RAW_ROW_BYTES));
-          uint4 o[4];
-          dequant32<FMT>(q, lut_l, a2, s2, o);
-          if constexpr (C::TMEM_A) {
-            const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
-                                    o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
-            tmem_st_32x32b_x16(t_lane + static_cast<uint32_t>(C::A_COL0 + stage * C::A_COLS + half * 16), v);
-            tmem_st_wait();
-            tc_fence_before_sync();
-          } else {
-            uint8_t* a = sA + stage * C::A_STAGE_BYTES;
+        const int nraw = (ksteps + 1) / 2;
+        for (int j = static_cast<int>((group - gr) & 1); j < nraw; j += 2) {
+          const int64_t rg = gr + j;
+          const int rs = static_cast<int>(rg % C::RAW_STAGES);
+          const uint32_t rph = static_cast<uint32_t>(rg / C::RAW_STAGES) & 1u;
+          uint64_t a2[2] = {0, 0};
+          uint32_t s2[2] = {0, 0};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
-            fence_proxy_async_smem();
+          for (int h = 0; h < 2; ++h) {
+            const int ks = 2 * j + h;
+            if (ks < ksteps) {
+              if (FMT == E4B_NF4) a2[h] = dup_f32(__ldg(sc_nf4 + ks));
+              else s2[h] = e8m0_to_bf16x2(__ldg(sc_mx + 2 * ks + half));
+            }
           }
+          if (!mbar_wait(&raw_full[rs], rph, wctx, 301)) { ok = false; break; }
+          const uint8_t* raw = sRaw + rs * RAW_STAGE_BYTES;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int ks = 2 * j + h;
+            if (ks >= ksteps) break;
+            const int64_t sg = gs + ks;
+            const int st = static_cast<int>(sg % C::STAGES);
+            const uint32_t sph = static_cast<uint32_t>(sg / C::STAGES) & 1u;
+            if (!mbar_wait(&empty[st], sph ^ 1u, wctx, 302)) { ok = false; break; }
+            const uint4 q = *reinterpret_cast<const uint4*>(raw + swizzled_offset(raw_row, h * 2 + half, RAW_ROW_BYTES));
+            uint4 o[4];
+            dequant32<FMT>(q, lut_l, a2[h], s2[h], o);
+            if constexpr (C::TMEM_A) {
+              const uint32_t v[16] = {o[0].x, o[0].y, o[0].z, o[0].w, o[1].x, o[1].y, o[1].z, o[1].w,
+                                      o[2].x, o[2].y, o[2].z, o[2].w, o[3].x, o[3].y, o[3].z, o[3].w};
+              tmem_st_32x32b_x16(t_lane + static_cast<uint32_t>(C::A_COL0 + st * C::A_COLS + half * 16), v);
+              tmem_st_wait();
+              tc_fence_before_sync();
+            } else {
+              uint8_t* a = sA + st * C::A_STAGE_BYTES;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4*>(a + swizzled_offset(prow, half * 4 + i, 128)) = o[i];
+              fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[st]);
+          }
+          if (!ok) break;
           __syncwarp();
-          if (lane == 0) mbar_arrive(&a_full[stage]);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-          if ((ks & 1) == 1 || ks + 1 == ksteps) {
-            if (lane == 0) mbar_arrive(&raw_empty[rstage]);
-            if (++rstage == C::RAW_STAGES) { rstage = 0; rphase ^= 1u; }
-          }
+          if (lane == 0) mbar_arrive(&raw_empty[rs]);
         }
+        if (!ok) break;
+        if (lora && group == 0) {                  // the LoRA step: group 0 fills the stage after K
+          const int64_t sg = gs + ksteps;
+          const int st = static_cast<int>(sg % C::STAGES);
+          if (!mbar_wait(&empty[st], (static_cast<uint32_t>(sg / C::STAGES) & 1u) ^ 1u, wctx, 303)) {
+            ok = false;
+            break;
+          }
+          if (half == 0) {                           // warp-uniform
+            const uint16_t* bcol = p.lora_B + static_cast<int64_t>(t.e) * p.lora_rank * (2 * p.I) + wrow;
+            uint32_t v[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+              const uint32_t lo = (2 * jj < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * jj) * 2 * p.I) : 0u;
+              const uint32_t hi =
+                  (2 * jj + 1 < p.lora_rank) ? __ldg(bcol + static_cast<int64_t>(2 * jj + 1) * 2 * p.I) : 0u;
+              v[jj] = lo | (hi << 16);
+            }
+            if constexpr (C::TMEM_A) {
+              tmem_st_32x32b_x8(t_lane + static_cast<uint32_t>(C::A_COL0 + st * C::A_COLS), v);
+              tmem_st_wait();
+            } else {
+              uint8_t* a = sA + st * C::A_STAGE_BYTES;
+              *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 0, 128)) = make_uint4(v[0], v[1], v[2], v[3]);
+              *reinterpret_cast<uint4*>(a + swizzled_offset(prow, 1, 128)) = make_uint4(v[4], v[5], v[6], v[7]);
+            }
+          }
+          if constexpr (C::TMEM_A) tc_fence_before_sync();
+          else fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&a_full[st]);
+        }
+        gs += ksteps + (lora ? 1 : 0);
+        gr += nraw;
+        continue;                                  // the LoRA step is done above for these tiles
       }
       if (!ok) break;
       if (lora) {                                   // A rows of the LoRA step: B_e[:, wrow]^T, rank padded to 16
@@ -631,7 +681,7 @@ e4b_status launch_typed(const GroupedGemmLaunch& g, const CUtensorMap& tc, const
   const int64_t max_tiles = (active + (g.R + BN - 1) / BN) * prm.n_blocks;
   const int64_t sms = device_sm_count();
   const int grid = static_cast<int>(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, s>>>(tc, ta, tx, prm);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tc, ta, tx, prm);
   return cudaGetLastError() == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }
 

@@ -67,7 +67,7 @@ def test_decode_kernel_chunk_sizes(fmt, T):
     run_and_compare(w, T, tokens_per_tile=8)
 
 
-@pytest.mark.parametrize("tpt", [0, 8])
+@pytest.mark.parametrize("tpt", [0, 8, 192])
 @pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
 def test_lora_tiny_and_zero_b(fmt, tpt):
     w = Workload(f"lora_{fmt}", fmt, E=8, H=256, I=128, k=2, tokens=(96,), lora_rank=8, lora_alpha=16.0, seed=6)
