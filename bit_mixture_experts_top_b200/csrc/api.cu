@@ -112,8 +112,8 @@ struct KernelChoice {
 // Mean routed rows per active expert decides: a handful per expert -> the decode
 // kernel (weight-stream bound), with chunks of 8, 16 or 32 tokens so that one
 // decoded weight fragment serves up to 32 tokens; more -> the smallest tcgen05
-// tile that holds most experts' rows in one chunk (192, not 256, for prefill
-// keeps the weight tile in tensor memory).
+// tile that holds most experts' rows in one chunk, 256 for prefill (each
+// dequantised weight stage then feeds the most tokens).
 KernelChoice pick_kernel(const e4b_moe_desc& d, int32_t T) {
   const int64_t R = static_cast<int64_t>(T) * d.k;
   const int64_t active = R < d.E ? R : d.E;
@@ -126,7 +126,7 @@ KernelChoice pick_kernel(const e4b_moe_desc& d, int32_t T) {
   if (avg <= 16) return {false, 32};
   if (avg <= 48) return {false, 64};
   if (avg <= 96) return {false, 128};
-  return {false, 192};
+  return {false, 256};
 }
 
 template <typename T>
