@@ -46,25 +46,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest():
-    """Digest of the grouped-GEMM sources (both kernels): a recorded traffic figure is void once they change."""
+def source_digest(name):
+    """Digest of one kernel source: a recorded traffic figure is void once its kernel's source changes."""
     h = hashlib.sha256()
-    for name in ("grouped_gemm.cu", "skinny_gemm.cu"):
-        with open(os.path.join(ROOT, "bit_mixture_experts_top_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    with open(os.path.join(ROOT, "bit_mixture_experts_top_b200", "csrc", name), "rb") as f:
+        h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel_tag, workload):
-    """DRAM bytes per launch of the kernel from the committed ncu summary, if it still matches the source
-    and was taken on this workload."""
+def recorded_traffic(kernel_tag, workload, source):
+    """DRAM bytes per launch of the kernel from the committed ncu summary, if it still matches the kernel's
+    source file and was taken on this workload."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_tag)
-    if not e or e.get("source_digest") != source_digest() or not e.get("workload", "").startswith(workload + " "):
+    if not e or e.get("source") != source or e.get("source_digest") != source_digest(source) \
+            or not e.get("workload", "").startswith(workload + " "):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -392,7 +392,8 @@ def bench_e4b(args, world, rank, local):
                                 "SwiGLU)" if decode_kernel else
                                 "grouped_gemm gate_up (tcgen05, dequant to tensor memory, SwiGLU)"),
                      **roof, "peak_kind": peak_kind,
-                     "traffic": recorded_traffic("gate_up", f"{args.workload} T={T}"),
+                     "traffic": recorded_traffic("gate_up", f"{args.workload} T={T}",
+                                                 "skinny_gemm.cu" if decode_kernel else "grouped_gemm.cu"),
                      "avg_launch_ms": gu_ms},
         "kernels": {"gate_up_ms": gu_ms, "down_ms": dn_ms, **small_ms,
                     "down_gbs": dn_bytes / (dn_ms * 1e-3) / 1e9,
