@@ -502,20 +502,28 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         // group takes code stage j of the tile when gr + j has its parity
         const int ksteps = p.K / ATOM_K;
         const int nraw = (ksteps + 1) / 2;
-        for (int j = static_cast<int>((group - gr) & 1); j < nraw; j += 2) {
-          const int64_t rg = gr + j;
-          const int rs = static_cast<int>(rg % C::RAW_STAGES);
-          const uint32_t rph = static_cast<uint32_t>(rg / C::RAW_STAGES) & 1u;
-          uint64_t a2[2] = {0, 0};
-          uint32_t s2[2] = {0, 0};
+        // scales of code stage j (two MMA stages), loaded one owned stage ahead
+        auto load_scales = [&](int j, uint64_t (&a2)[2], uint32_t (&s2)[2]) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int ks = 2 * j + h;
-            if (ks < ksteps) {
+            if (j < nraw && ks < ksteps) {
               if (FMT == E4B_NF4) a2[h] = dup_f32(__ldg(sc_nf4 + ks));
               else s2[h] = e8m0_to_bf16x2(__ldg(sc_mx + 2 * ks + half));
             }
           }
+        };
+        const int j0 = static_cast<int>((group - gr) & 1);
+        uint64_t a2n[2] = {0, 0};
+        uint32_t s2n[2] = {0, 0};
+        load_scales(j0, a2n, s2n);
+        for (int j = j0; j < nraw; j += 2) {
+          const int64_t rg = gr + j;
+          const int rs = static_cast<int>(rg % C::RAW_STAGES);
+          const uint32_t rph = static_cast<uint32_t>(rg / C::RAW_STAGES) & 1u;
+          const uint64_t a2[2] = {a2n[0], a2n[1]};
+          const uint32_t s2[2] = {s2n[0], s2n[1]};
+          load_scales(j + 2, a2n, s2n);
           if (!mbar_wait(&raw_full[rs], rph, wctx, 301)) { ok = false; break; }
           const uint8_t* raw = sRaw + rs * RAW_STAGE_BYTES;
 #pragma unroll
