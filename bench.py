@@ -193,6 +193,46 @@ def bench_reference(args, world, rank):
     return 0
 
 
+class Replicas:
+    """Process-group plumbing of the replicas run: one process per GPU, no data exchange;
+    a barrier around the timed region and the max over ranks of every time.  NCCL on GPUs,
+    gloo for the CPU tests of this logic; world == 1 needs no process group."""
+
+    def __init__(self, world, rank, backend="nccl", device=None, timeout_s=120):
+        import torch
+        self.world, self.rank, self.device = world, rank, device
+        self.dist = world > 1
+        if self.dist:
+            import datetime
+            import torch.distributed as tdist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+        self._torch = torch
+
+    def barrier(self):
+        if self.dist:
+            self._torch.distributed.barrier()
+
+    def max_over_ranks(self, v):
+        if not self.dist:
+            return v
+        t = self._torch.tensor([v], dtype=self._torch.float64, device=self.device)
+        self._torch.distributed.all_reduce(t, op=self._torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def whole_job_rate(self, units_per_rank, ms_max):
+        """Units every rank processed per second of the slowest rank (weak scaling)."""
+        return self.world * units_per_rank / (ms_max * 1e-3)
+
+    def emit(self, line):
+        if self.rank == 0:
+            print(json.dumps(line), flush=True)
+
+    def close(self):
+        if self.dist:
+            self._torch.distributed.destroy_process_group()
+
+
 def bench_e4b(args, world, rank, local):
     import torch
     from bit_mixture_experts_top_b200 import e4b, layer
@@ -200,24 +240,11 @@ def bench_e4b(args, world, rank, local):
 
     dist = world > 1
     if dist:
-        import datetime
-        import torch.distributed as tdist
         torch.cuda.set_device(local)
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local if dist else 0)
     torch.cuda.set_device(dev)
-
-    def barrier():
-        if dist:
-            torch.distributed.barrier()
-
-    def max_over_ranks(v):
-        if not dist:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    rep = Replicas(world, rank, "nccl", dev)
+    barrier, max_over_ranks = rep.barrier, rep.max_over_ranks
 
     w = WORKLOADS[args.workload]
     T = args.tokens
@@ -379,7 +406,7 @@ def bench_e4b(args, world, rank, local):
         roof = {"bound": "hbm", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "algorithmic_bytes_per_launch": gu_bytes}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    value = world * T / (ms_per_step * 1e-3)
+    value = rep.whole_job_rate(T, ms_per_step)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -399,7 +426,7 @@ def bench_e4b(args, world, rank, local):
                     "down_gbs": dn_bytes / (dn_ms * 1e-3) / 1e9,
                     "layer_weight_gbs": layer_weight_bytes / (ms_per_step * 1e-3) / 1e9,
                     "touched_experts": touched},
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": rep.whole_job_rate(T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "path": "layer.HostForward.run: pinned host inputs -> device -> forward -> pinned host output, "
                         "one CUDA graph replay and a synchronize per step"},
@@ -414,10 +441,8 @@ def bench_e4b(args, world, rank, local):
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{what} ({ne} experts decoded in fp64), "
                                           f"timed twice, {dt:.1f} s per forward"}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if dist:
-        torch.distributed.destroy_process_group()
+    rep.emit(line)
+    rep.close()
     return 0
 
 
