@@ -14,6 +14,7 @@ Recipe (all streams keyed by ``seed`` and a tensor name):
   test (and independently by the oracle);
 * LoRA: A ~ N(0, 1/r), B ~ N(0, 0.01) in bf16 (the second parameter is read
   as a standard deviation);
+* gpt-oss epilogue biases: fp32 N(0, std), std chosen per test;
 * skewed routing: logits log p_e + Gumbel(0, 1) with p_e proportional to
   rank**-s over a seeded permutation of the experts, so a top-k pick is a
   Gumbel-top-k draw without replacement and expert load is Zipf(s) skewed.
@@ -40,6 +41,11 @@ def to_bf16_bits(a):
 
 def normal_bf16(shape, std, seed, name):
     return to_bf16_bits(rng(seed, name).standard_normal(shape, dtype=np.float32) * np.float32(std))
+
+
+def normal_f32(shape, std, seed, name):
+    """fp32 N(0, std) values (biases of the gpt-oss epilogue)."""
+    return rng(seed, name).standard_normal(shape, dtype=np.float32) * np.float32(std)
 
 
 def expert_normal_f32(e, N, K, std, seed, name):

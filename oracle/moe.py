@@ -13,6 +13,10 @@ Sources on the pages:
 * "experts4bit-qlora" package page, "What it does": the experts of a layer are
   one fused three-dimensional parameter ``[E, ...]``.
 * Examples on the pages use LoRA rank r = 8 and alpha = 16.
+* "How do I train and serve MoE models released in MXFP4 (gpt-oss,
+  DeepSeek-V4)?", "Why it happens": gpt-oss experts add per-expert biases,
+  interleaved gate/up rows and a clamped GLU; "Which project solves it": the
+  gpt-oss module handles the biases, the de-interleave and the clamped GLU.
 
 The forward, in the pages' order and with every product in fp64:
 
@@ -33,6 +37,16 @@ Readings where the pages are silent:
   named on the MXFP4 page as a gpt-oss peculiarity, outside the stock epilogue).
 * One LoRA adapter per expert on the fused gate_up output: A_e [H, r],
   B_e [r, 2I].
+* gpt-oss epilogue (the pages name its three parts but print no formula or
+  constant):
+  - interleaved rows put gate i at stored row 2i and up i at row 2i + 1; they
+    are de-interleaved once, at load, into [gate | up] (:func:`deinterleave_rows`);
+  - biases b_gu [E, 2I] (in [gate | up] order) and b_dn [E, H] are added to G
+    before the activation and to Y before the combine, so the combine weights
+    scale the down bias too;
+  - clamped GLU with parameters alpha, limit and up offset beta:
+    g = min(gate, limit), u = clamp(up, -limit, limit),
+    h = g * sigmoid(alpha * g) * (u + beta).
 """
 import numpy as np
 
@@ -63,9 +77,34 @@ def silu(z):
         return z / (1.0 + np.exp(-z))
 
 
+def clamped_glu(gate, up, alpha, limit, beta):
+    """gpt-oss clamped GLU in fp64: min(gate, limit) * sigmoid(alpha * .) * (clamp(up, +-limit) + beta)."""
+    g = np.minimum(gate, limit)
+    u = np.clip(up, -limit, limit)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-alpha * g)) * (u + beta)
+
+
+def deinterleave_rows(stack, E, I):
+    """[E, 2I, ...] with gate i at row 2i and up i at row 2i + 1  ->  [E, 2I, ...] as [gate | up].
+
+    A pure row permutation of whatever each row holds (packed codes, scale
+    bytes or one bias value), so it applies unchanged to every tensor of the
+    gate_up stack.
+    """
+    a = np.asarray(stack)
+    rows = a.reshape(E, 2 * I, -1)
+    return np.concatenate([rows[:, 0::2], rows[:, 1::2]], axis=1).reshape(a.shape)
+
+
 def moe_forward(x_bits, logits_bits, k, fmt, E, H, I, gu_codes, gu_scales, dn_codes, dn_scales,
-                lora_A_bits=None, lora_B_bits=None, lora_scale=0.0):
-    """Layer forward.  x: bf16 bits [T, H]; logits: bf16 bits [T, E].  Returns (out fp64 [T, H], route dict)."""
+                lora_A_bits=None, lora_B_bits=None, lora_scale=0.0, gu_bias=None, dn_bias=None, glu=None):
+    """Layer forward.  x: bf16 bits [T, H]; logits: bf16 bits [T, E].  Returns (out fp64 [T, H], route dict).
+
+    gu_bias [E, 2I] / dn_bias [E, H] (fp32, or None for no bias) and
+    glu = (alpha, limit, beta) select the gpt-oss epilogue; glu None is the
+    stock SwiGLU silu(gate) * up.
+    """
     x = bf16_bits_to_f64(np.asarray(x_bits, dtype=np.uint16)).reshape(-1, H)
     T = x.shape[0]
     r = route(np.asarray(logits_bits, dtype=np.uint16).reshape(T, E), k)
@@ -88,9 +127,16 @@ def moe_forward(x_bits, logits_bits, k, fmt, E, H, I, gu_codes, gu_scales, dn_co
         G = Xe @ Wgu.T
         if lora:
             G = G + lora_scale * ((Xe @ A[e]) @ B[e])
-        h = silu(G[:, :I]) * G[:, I:]
+        if gu_bias is not None:
+            G = G + np.asarray(gu_bias, dtype=np.float64).reshape(E, 2 * I)[e]
+        if glu is None:
+            h = silu(G[:, :I]) * G[:, I:]
+        else:
+            h = clamped_glu(G[:, :I], G[:, I:], *glu)
         Wdn = decode_expert(fmt, dn_codes, dn_scales, e, H, I)         # [H, I]
         y_sorted[lo:hi] = h @ Wdn.T
+        if dn_bias is not None:
+            y_sorted[lo:hi] += np.asarray(dn_bias, dtype=np.float64).reshape(E, H)[e]
     out = np.zeros((T, H), dtype=np.float64)             # step 4: combine, j ascending
     for j in range(k):
         pos = r["slot_pos"][np.arange(T) * k + j]

@@ -3,7 +3,10 @@
 Routing is checked against a per-token brute-force sort; the grouped forward
 against a per-token dense loop written independently here, against the
 textbook dense SwiGLU FFN (E = 1, k = 1), against token permutation and
-against a zero LoRA B.
+against a zero LoRA B.  The gpt-oss epilogue (biases, clamped GLU,
+de-interleave) is checked by its reductions (SwiGLU, relu limit), its
+saturation points, a shared down bias that shifts every token by itself,
+zero gate_up weights that leave only the bias, and a per-token loop.
 """
 import math
 
@@ -170,3 +173,129 @@ def test_synth_is_deterministic_and_per_expert():
     top = int(np.argmax(r["counts"]))
     first = np.mean(r["ids"][:, 0] == top)     # first Gumbel-top-k draw follows p_e: ~0.226 for rank 1
     assert 0.20 < first < 0.25
+
+
+# ---------------------------------------------------------------- gpt-oss epilogue
+
+GPTOSS_GLU = (1.702, 7.0, 1.0)    # alpha, limit, up offset of the public gpt-oss release
+
+
+def test_clamped_glu_reduces_to_silu_times_up():
+    g = np.random.default_rng(11)
+    gate, up = g.standard_normal(1000) * 5, g.standard_normal(1000) * 5
+    assert np.array_equal(moe.clamped_glu(gate, up, 1.0, np.inf, 0.0), moe.silu(gate) * up)
+
+
+def test_clamped_glu_limits_and_saturation():
+    a, L, b = GPTOSS_GLU
+    up = np.array([-3.0, 0.5, 2.0])
+    # large alpha: g * sigmoid(alpha g) -> relu(g)
+    gate = np.array([-2.0, -0.5, 0.5, 3.0])
+    hb = moe.clamped_glu(gate[:, None], up[None, :], 1e4, L, b)
+    assert np.array_equal(hb, np.maximum(gate, 0.0)[:, None] * (up + b)[None, :])
+    # gate clamps from above only; up clamps on both sides
+    h = lambda gt, u: moe.clamped_glu(np.float64(gt), np.float64(u), a, L, b)
+    assert h(L + 0.25, 1.0) == h(L, 1.0) == h(1e6, 1.0)
+    assert h(-L - 5.0, 1.0) != h(-L, 1.0)
+    assert h(2.0, L + 3.0) == h(2.0, L) and h(2.0, -L - 3.0) == h(2.0, -L)
+    assert h(2.0, L - 1.0) != h(2.0, L)
+    # the up offset: u = -beta zeroes the product; gate 0 zeroes it too
+    assert h(2.0, -b) == 0.0 and h(0.0, 3.0) == 0.0
+    # sigmoid(alpha g) at g = 0 is 1/2: slope of g -> h at 0 is (u + b) / 2
+    eps = 1e-7
+    assert abs(h(eps, 1.0) / eps - (1.0 + b) / 2) < 1e-6
+
+
+def test_deinterleave_rows_puts_even_rows_first():
+    E, I, R = 3, 5, 4
+    gate = np.arange(E * I * R).reshape(E, I, R)
+    up = -1 - gate
+    inter = np.empty((E, 2 * I, R), dtype=np.int64)
+    for e in range(E):
+        for i in range(I):
+            inter[e, 2 * i], inter[e, 2 * i + 1] = gate[e, i], up[e, i]
+    out = moe.deinterleave_rows(inter.reshape(-1), E, I).reshape(E, 2 * I, R)
+    assert np.array_equal(out[:, :I], gate) and np.array_equal(out[:, I:], up)
+    bias = inter[:, :, 0]                                   # one value per row
+    assert np.array_equal(moe.deinterleave_rows(bias, E, I), np.concatenate([gate[:, :, 0], up[:, :, 0]], 1))
+
+
+def _dense_loop_gptoss(fmt, x, logits, k, E, H, I, gu, dn, bgu, bdn, glu):
+    """Per token, per choice, with the biases and the clamped GLU written out element by element."""
+    a, L, b = glu
+    xf = bf16.bf16_bits_to_f64(x)
+    lf = bf16.bf16_bits_to_f64(logits)
+    out = np.zeros((xf.shape[0], H))
+    for t in range(xf.shape[0]):
+        ids = _brute_topk(lf[t], k)
+        z = np.array([lf[t, e] for e in ids])
+        w = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+        for j, e in enumerate(ids):
+            g = _decode(fmt, gu[0], gu[1], e, 2 * I, H) @ xf[t] + bgu[e]
+            h = np.empty(I)
+            for i in range(I):
+                gt, u = min(g[i], L), max(-L, min(g[I + i], L))
+                h[i] = gt / (1.0 + math.exp(-a * gt)) * (u + b)
+            out[t] += w[j] * (_decode(fmt, dn[0], dn[1], e, H, I) @ h + bdn[e])
+    return out
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+def test_forward_gptoss_epilogue_equals_dense_loop(fmt):
+    E, H, I, k, T = 4, 64, 64, 2, 12
+    gu, dn = _tiny_layer(fmt, E, H, I, seed=12)
+    x = synth.normal_bf16((T, H), 1.0, 12, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 12, "logits")
+    bgu = synth.normal_f32((E, 2 * I), 0.5, 12, "bgu")
+    bdn = synth.normal_f32((E, H), 0.5, 12, "bdn")
+    glu = GPTOSS_GLU if fmt == "mxfp4" else (1.702, 0.1, 1.0)    # NF4 outputs are small: clamp lower
+    out, _ = moe.moe_forward(x, logits, k, fmt, E, H, I, gu[0], gu[1], dn[0], dn[1],
+                             gu_bias=bgu, dn_bias=bdn, glu=glu)
+    ref = _dense_loop_gptoss(fmt, x, logits, k, E, H, I, gu, dn, bgu, bdn, glu)
+    assert np.allclose(out, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
+
+
+def test_forward_shared_down_bias_shifts_every_token_by_it():
+    E, H, I, k, T = 8, 64, 64, 3, 20
+    gu, dn = _tiny_layer("nf4", E, H, I, seed=13)
+    x = synth.normal_bf16((T, H), 1.0, 13, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 13, "logits")
+    b = synth.normal_f32((H,), 1.0, 13, "b")
+    base, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1], glu=GPTOSS_GLU)
+    shifted, _ = moe.moe_forward(x, logits, k, "nf4", E, H, I, gu[0], gu[1], dn[0], dn[1],
+                                 dn_bias=np.tile(b, (E, 1)), glu=GPTOSS_GLU)
+    assert np.allclose(shifted - base, np.broadcast_to(b, base.shape), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+def test_forward_zero_gate_up_weights_leave_the_bias(fmt):
+    E, H, I, T = 1, 64, 64, 5
+    _, dn = _tiny_layer(fmt, E, H, I, seed=14)
+    if fmt == "mxfp4":
+        gu = (np.zeros(2 * I * H // 2, np.uint8), np.full(2 * I * H // 32, 127, np.uint8))
+    else:
+        gu = nf4.quantize_nf4(np.zeros((E, 2 * I, H), np.float32))
+    x = synth.normal_bf16((T, H), 1.0, 14, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 14, "logits")
+    bgu = synth.normal_f32((E, 2 * I), 4.0, 14, "bgu")
+    out, _ = moe.moe_forward(x, logits, 1, fmt, E, H, I, gu[0], gu[1], dn[0], dn[1], gu_bias=bgu, glu=GPTOSS_GLU)
+    Wd = _decode(fmt, dn[0], dn[1], 0, H, I)
+    h = moe.clamped_glu(bgu[0, :I].astype(np.float64), bgu[0, I:].astype(np.float64), *GPTOSS_GLU)
+    assert np.allclose(out, np.tile(Wd @ h, (T, 1)), rtol=1e-13, atol=1e-13 * np.abs(Wd @ h).max())
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+def test_deinterleave_restores_released_gate_up_tensors(fmt):
+    E, H, I = 4, 64, 64
+    gu, _ = _tiny_layer(fmt, E, H, I, seed=15)
+    bgu = synth.normal_f32((E, 2 * I), 0.5, 15, "bgu")
+    # the released layout: rows alternate gate i, up i (codes, scale rows and biases alike)
+    codes = gu[0].reshape(E, 2 * I, H // 2)
+    scales = np.asarray(gu[1]).reshape(E, 2 * I, -1)
+    ic, isc, ib = np.empty_like(codes), np.empty_like(scales), np.empty_like(bgu)
+    ic[:, 0::2], ic[:, 1::2] = codes[:, :I], codes[:, I:]
+    isc[:, 0::2], isc[:, 1::2] = scales[:, :I], scales[:, I:]
+    ib[:, 0::2], ib[:, 1::2] = bgu[:, :I], bgu[:, I:]
+    assert np.array_equal(moe.deinterleave_rows(ic, E, I), codes)
+    assert np.array_equal(moe.deinterleave_rows(isc, E, I), scales)
+    assert np.array_equal(moe.deinterleave_rows(ib, E, I), bgu)
