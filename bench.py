@@ -255,7 +255,7 @@ def bench_e4b(args, world, rank, local):
     out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
     ws = lay.workspace(T, dev)
     args_fwd = (lay.desc, T, x, lg, lay.gate_up.codes, lay.gate_up.scales, lay.down.codes, lay.down.scales,
-                lay.lora_A, lay.lora_B, out, ws)
+                lay.lora_A, lay.lora_B, lay.gu_bias, lay.dn_bias, out, ws)
 
     def forward():
         e4b.e4b_moe_forward(*args_fwd)

@@ -2,6 +2,7 @@
 // sequence of the layer forward (route -> gather -> gate_up -> down -> combine).
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstring>
 
 #include "e4b.h"
@@ -91,7 +92,10 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (d->E < 1 || d->E > kMaxExperts || d->k < 1 || d->k > d->E || d->k > kMaxTopK) return E4B_ERR_UNSUPPORTED;
   if (d->H < 64 || d->H % 64 != 0 || d->I < 64 || d->I % 64 != 0) return E4B_ERR_UNSUPPORTED;
   if (d->format != E4B_NF4 && d->format != E4B_MXFP4) return E4B_ERR_UNSUPPORTED;
-  if (d->act != E4B_ACT_SWIGLU) return E4B_ERR_UNSUPPORTED;
+  if (d->act != E4B_ACT_SWIGLU && d->act != E4B_ACT_CLAMPED_GLU) return E4B_ERR_UNSUPPORTED;
+  if (d->act == E4B_ACT_CLAMPED_GLU &&
+      (!std::isfinite(d->glu_alpha) || !std::isfinite(d->glu_beta) || !(d->glu_limit > 0.0f)))
+    return E4B_ERR_INVALID_ARG;
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
   const int tpt = d->tokens_per_tile;
   if (tpt == 8 && !(skinny_gemm_supported(d->H, d->format) && skinny_gemm_supported(d->I, d->format)))
@@ -169,6 +173,19 @@ e4b_status e4b_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_
              : E4B_ERR_CUDA;
 }
 
+e4b_status e4b_deinterleave_rows(const void* in, void* out, int32_t E, int32_t I, int64_t row_bytes,
+                                 e4b_stream stream) {
+  if (E < 0 || I < 0 || row_bytes < 0) return E4B_ERR_INVALID_ARG;
+  const int64_t bytes = static_cast<int64_t>(E) * 2 * I * row_bytes;
+  if (bytes == 0) return E4B_OK;
+  if (!in || !out) return E4B_ERR_INVALID_ARG;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+  if (a < b + static_cast<uintptr_t>(bytes) && b < a + static_cast<uintptr_t>(bytes)) return E4B_ERR_INVALID_ARG;
+  return launch_deinterleave_rows(in, out, E, I, row_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? E4B_OK
+             : E4B_ERR_CUDA;
+}
+
 e4b_status e4b_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, e4b_stream stream) {
   if (n < 0 || n % 64 != 0) return E4B_ERR_INVALID_ARG;
   if (n == 0) return E4B_OK;
@@ -237,7 +254,8 @@ e4b_status e4b_moe_workspace_region(const e4b_moe_desc* d, int32_t T, int32_t re
 static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d, int32_t T, const uint16_t* x,
                              const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
                              const uint8_t* dn_codes, const void* dn_scales, const uint16_t* lora_A,
-                             const uint16_t* lora_B, uint16_t* out, void* ws, size_t ws_bytes, e4b_stream stream) {
+                             const uint16_t* lora_B, const float* gu_bias, const float* dn_bias, uint16_t* out,
+                             void* ws, size_t ws_bytes, e4b_stream stream) {
   const e4b_status v = validate_desc(d, T);
   if (v != E4B_OK) return v;
   if (first < E4B_STAGE_ROUTE || last > E4B_STAGE_COMBINE || first > last) return E4B_ERR_INVALID_ARG;
@@ -252,6 +270,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         !aligned(gu_scales, 16) || !aligned(dn_scales, 16))
       return E4B_ERR_INVALID_ARG;
     if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 2))) return E4B_ERR_INVALID_ARG;
+    if ((gu_bias && !aligned(gu_bias, 4)) || (dn_bias && !aligned(dn_bias, 4))) return E4B_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const KernelChoice kc = pick_kernel(*d, T);
@@ -284,6 +303,10 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   g.chunk_off = b.chunk_off;
   g.status = b.status;
   g.wait_limit_ns = kWaitLimitNs;
+  g.glu = d->act;
+  g.glu_alpha = d->glu_alpha;
+  g.glu_limit = d->glu_limit;
+  g.glu_beta = d->glu_beta;
 
   for (int32_t stage = first; stage <= last; ++stage) {
     switch (stage) {
@@ -306,6 +329,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.xa = xa;
         g.lora_B = lora_B;
         g.lora_rank = d->lora_rank;
+        g.bias = gu_bias;
         g.out = h;
         const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
@@ -321,6 +345,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.xa = nullptr;
         g.lora_B = nullptr;
         g.lora_rank = 0;
+        g.bias = dn_bias;
         g.out = y;
         const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
@@ -336,19 +361,20 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
 
 e4b_status e4b_moe_forward(const e4b_moe_desc* d, int32_t T, const uint16_t* x, const uint16_t* logits,
                            const uint8_t* gu_codes, const void* gu_scales, const uint8_t* dn_codes,
-                           const void* dn_scales, const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* out,
-                           void* ws, size_t ws_bytes, e4b_stream stream) {
+                           const void* dn_scales, const uint16_t* lora_A, const uint16_t* lora_B,
+                           const float* gu_bias, const float* dn_bias, uint16_t* out, void* ws, size_t ws_bytes,
+                           e4b_stream stream) {
   return run_stages(E4B_STAGE_ROUTE, E4B_STAGE_COMBINE, d, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales,
-                    lora_A, lora_B, out, ws, ws_bytes, stream);
+                    lora_A, lora_B, gu_bias, dn_bias, out, ws, ws_bytes, stream);
 }
 
 e4b_status e4b_moe_forward_stage(int32_t stage, const e4b_moe_desc* d, int32_t T, const uint16_t* x,
                                  const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
                                  const uint8_t* dn_codes, const void* dn_scales, const uint16_t* lora_A,
-                                 const uint16_t* lora_B, uint16_t* out, void* ws, size_t ws_bytes,
-                                 e4b_stream stream) {
-  return run_stages(stage, stage, d, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, out,
-                    ws, ws_bytes, stream);
+                                 const uint16_t* lora_B, const float* gu_bias, const float* dn_bias, uint16_t* out,
+                                 void* ws, size_t ws_bytes, e4b_stream stream) {
+  return run_stages(stage, stage, d, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias,
+                    dn_bias, out, ws, ws_bytes, stream);
 }
 
 e4b_status e4b_device_status(void* ws, e4b_stream stream) {

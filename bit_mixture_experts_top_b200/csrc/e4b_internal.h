@@ -56,6 +56,8 @@ cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, in
                                  cudaStream_t s);
 
 cudaError_t launch_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, cudaStream_t s);
+cudaError_t launch_deinterleave_rows(const void* in, void* out, int32_t E, int32_t I, int64_t row_bytes,
+                                     cudaStream_t s);
 
 // x_sorted[r] = x[sorted_slot[r] / k]; with LoRA also xa[r, j] = bf16(scale * x . A_e[:, j]) (j < r, zeros to 64).
 cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, const int32_t* sorted_slot,
@@ -85,6 +87,9 @@ struct GroupedGemmLaunch {
   void* out;                // mode 0: bf16 [R, I]; mode 1: fp32 [R, H]
   int32_t* status;
   uint64_t wait_limit_ns;
+  const float* bias;        // mode 0: [E, 2I] ([gate | up]); mode 1: [E, H]; null = none
+  int32_t glu;              // E4B_ACT_SWIGLU / E4B_ACT_CLAMPED_GLU (mode 0)
+  float glu_alpha, glu_limit, glu_beta;
 };
 e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 

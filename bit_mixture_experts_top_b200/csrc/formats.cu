@@ -136,6 +136,44 @@ int grid_for(int64_t work_items, int threads, int per_sm) {
 
 }  // namespace
 
+// gpt-oss gate_up de-interleave ("How do I train and serve MoE models released
+// in MXFP4 ...?", "Why it happens": interleaved gate/up rows; "Which project
+// solves it": the gpt-oss module de-interleaves them): row n of expert e in
+// the output is input row 2n (gate, n < I) or 2(n - I) + 1 (up).  A plain row
+// gather, moved in the widest word the row size and the pointers allow.
+template <typename W>
+__global__ void __launch_bounds__(256) deinterleave_rows_kernel(const W* __restrict__ in, W* __restrict__ out,
+                                                                int64_t rows, int32_t I, int64_t words_per_row) {
+  const int64_t total = rows * words_per_row;
+  for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < total;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = u / words_per_row, w = u - row * words_per_row;
+    const int64_t e = row / (2 * I), n = row - e * 2 * I;
+    const int64_t src = e * 2 * I + (n < I ? 2 * n : 2 * (n - I) + 1);
+    out[u] = __ldg(in + src * words_per_row + w);
+  }
+}
+
+cudaError_t launch_deinterleave_rows(const void* in, void* out, int32_t E, int32_t I, int64_t row_bytes,
+                                     cudaStream_t s) {
+  const int64_t rows = static_cast<int64_t>(E) * 2 * I;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out);
+  if (rows == 0 || row_bytes == 0) return cudaSuccess;
+  if (row_bytes % 16 == 0 && a % 16 == 0) {
+    const int64_t wpr = row_bytes / 16;
+    deinterleave_rows_kernel<uint4><<<grid_for(rows * wpr, 256, 8), 256, 0, s>>>(
+        static_cast<const uint4*>(in), static_cast<uint4*>(out), rows, I, wpr);
+  } else if (row_bytes % 4 == 0 && a % 4 == 0) {
+    const int64_t wpr = row_bytes / 4;
+    deinterleave_rows_kernel<uint32_t><<<grid_for(rows * wpr, 256, 8), 256, 0, s>>>(
+        static_cast<const uint32_t*>(in), static_cast<uint32_t*>(out), rows, I, wpr);
+  } else {
+    deinterleave_rows_kernel<uint8_t><<<grid_for(rows * row_bytes, 256, 8), 256, 0, s>>>(
+        static_cast<const uint8_t*>(in), static_cast<uint8_t*>(out), rows, I, row_bytes);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n, uint16_t* out,
                                  cudaStream_t s) {
   const int64_t units = n / 8;

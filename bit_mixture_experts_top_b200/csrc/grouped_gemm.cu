@@ -7,8 +7,12 @@
 // experts4bit-qlora table of the index: ExpertsLoRA's per-expert low-rank
 // delta before the activation):
 //
-//   mode 0 (gate_up): G = X_e W_gu[e]^T (+ xa_e B_e), h = silu(G_gate) * G_up -> bf16 [R, I]
-//   mode 1 (down)   : Y = h_e W_dn[e]^T                                       -> fp32 [R, H]
+//   mode 0 (gate_up): G = X_e W_gu[e]^T (+ xa_e B_e) (+ b_gu[e]), h = act(G_gate, G_up) -> bf16 [R, I]
+//   mode 1 (down)   : Y = h_e W_dn[e]^T (+ b_dn[e])                           -> fp32 [R, H]
+//
+// act is silu(gate) * up, or the gpt-oss clamped GLU with per-expert biases
+// ("How do I train and serve MoE models released in MXFP4 (gpt-oss,
+// DeepSeek-V4)?", "Why it happens"); see Epilogue in e4b_device.cuh.
 //
 // B200 design.  The weights are the UMMA M operand (128 rows per tile; in
 // tensor memory for decode-sized tiles, in shared memory for prefill tiles)
@@ -111,6 +115,7 @@ struct Params {
   void* out;
   int32_t* status;
   uint64_t wait_limit_ns;
+  Epilogue ep;            // biases and activation
   float lut[16];          // NF4 levels
 };
 
@@ -639,22 +644,24 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
         if (MODE == 0) {
           const int f = 64 * t.nb + 16 * q + (lane & 15);
           __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+          // lanes 0-15 hold gate rows, lanes 16-31 the matching up rows
+          const float bv = p.ep.bias ? __ldg(p.ep.bias + static_cast<int64_t>(t.e) * 2 * p.I + (lane < 16 ? 0 : p.I) + f)
+                                     : 0.f;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            const float v = __uint_as_float(r[j]);
+            const float v = __uint_as_float(r[j]) + bv;
             const float u = __shfl_xor_sync(kFull, v, 16);
-            if (lane < 16 && c0 + j < t.rows) {
-              const float sg = __fdividef(v, 1.0f + __expf(-v));
-              h[static_cast<int64_t>(t.row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(sg * u);
-            }
+            if (lane < 16 && c0 + j < t.rows)
+              h[static_cast<int64_t>(t.row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(expert_act(p.ep, v, u));
           }
         } else {
           const int n = BM * t.nb + 32 * q + lane;
           float* y = reinterpret_cast<float*>(p.out);
           if (n < p.N) {
+            const float bv = p.ep.bias ? __ldg(p.ep.bias + static_cast<int64_t>(t.e) * p.N + n) : 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (c0 + j < t.rows) y[static_cast<int64_t>(t.row0 + c0 + j) * p.N + n] = __uint_as_float(r[j]);
+              if (c0 + j < t.rows) y[static_cast<int64_t>(t.row0 + c0 + j) * p.N + n] = __uint_as_float(r[j]) + bv;
           }
         }
       }
@@ -763,6 +770,7 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.out = g.out;
   prm.status = g.status;
   prm.wait_limit_ns = g.wait_limit_ns;
+  prm.ep = Epilogue{g.bias, g.mode == 0 ? g.glu : E4B_ACT_SWIGLU, g.glu_alpha, g.glu_limit, g.glu_beta};
   for (int i = 0; i < 16; ++i) prm.lut[i] = nf4_table().level[i];
   switch (BN) {
     case 32: return dispatch_fmt_mode<32>(g, tc, ta, tx, prm, s);

@@ -21,7 +21,8 @@
 //  * mode 0 (gate_up): rows are gate columns 64nb..64nb+63 and the matching up
 //    columns I+64nb..; MMA tile t pairs gate rows 8t..8t+7 with up rows
 //    64+8t..64+8t+7, so one thread holds gate and up of the same (token,
-//    column) and applies SwiGLU in registers;
+//    column) and applies the biases and the activation (SwiGLU, or the
+//    gpt-oss clamped GLU) in registers;
 //  * mode 1 (down): output rows 128nb..128nb+127; tile t = rows 16t..16t+15.
 //
 // Warp roles (one CTA per SM, persistent):
@@ -102,6 +103,7 @@ struct SkParams {
   int32_t* status;
   uint32_t* counters;     // [2]: next unit, CTAs done (zero between launches)
   uint64_t wait_limit_ns;
+  Epilogue ep;            // biases and activation
   uint32_t level2[8];     // NF4: bf16 levels, two per word (level 2w low half)
 };
 
@@ -515,6 +517,20 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         la[2] = lora_pair(Be + col, rs, 2 * c + 8, p.lora_rank);
         la[3] = lora_pair(Be + p.I + col, rs, 2 * c + 8, p.lora_rank);
       }
+      // biases of the two output rows this lane finishes (gate/up pair, or rows n, n + 8)
+      float b_lo = 0.f, b_hi = 0.f;
+      if (fin && p.ep.bias) {
+        if (MODE == 0) {
+          const float* be = p.ep.bias + static_cast<int64_t>(un.e) * 2 * p.I + 64 * un.nb + 8 * t + rho;
+          b_lo = __ldg(be);
+          b_hi = __ldg(be + p.I);
+        } else {
+          const int n = SK_ROWS * un.nb + 16 * t + rho;
+          const float* be = p.ep.bias + static_cast<int64_t>(un.e) * p.N + n;
+          if (n < p.N) b_lo = __ldg(be);
+          if (n + 8 < p.N) b_hi = __ldg(be + 8);
+        }
+      }
 #pragma unroll
       for (int q = 0; q < TG; ++q) {
         if (!warp_wait(rempty, rph ^ 1u, wctx, 723)) { ok = false; break; }
@@ -551,9 +567,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
               if (tok0 + 2 * c + r < un.m) {
-                const float gt = v[r], up = v[2 + r];
-                const float sg = __fdividef(gt, 1.0f + __expf(-gt));
-                h[static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.I + col] = __float2bfloat16_rn(sg * up);
+                const float a = expert_act(p.ep, v[r] + b_lo, v[2 + r] + b_hi);
+                h[static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.I + col] = __float2bfloat16_rn(a);
               }
             }
           } else {
@@ -563,8 +578,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
             for (int r = 0; r < 2; ++r) {
               if (tok0 + 2 * c + r < un.m) {
                 float* yr = y + static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.N + n;
-                if (n < p.N) yr[0] = v[r];
-                if (n + 8 < p.N) yr[8] = v[2 + r];
+                if (n < p.N) yr[0] = v[r] + b_lo;
+                if (n + 8 < p.N) yr[8] = v[2 + r] + b_hi;
               }
             }
           }
@@ -641,6 +656,7 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.chunk_off = g.chunk_off;
   prm.out = g.out;
   prm.status = g.status;
+  prm.ep = Epilogue{g.bias, g.mode == 0 ? g.glu : E4B_ACT_SWIGLU, g.glu_alpha, g.glu_limit, g.glu_beta};
   prm.counters = reinterpret_cast<uint32_t*>(g.status) + 8 + 2 * g.mode;
   prm.wait_limit_ns = g.wait_limit_ns;
   const Nf4Table& t = nf4_table();

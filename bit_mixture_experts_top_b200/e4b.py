@@ -18,7 +18,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "e4b.h")
 
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_UNSUPPORTED, E4B_ERR_CUDA, E4B_ERR_TIMEOUT = range(5)
 E4B_NF4, E4B_MXFP4 = 0, 1
-E4B_ACT_SWIGLU = 0
+E4B_ACT_SWIGLU, E4B_ACT_CLAMPED_GLU = 0, 1
 E4B_STAGE_ROUTE, E4B_STAGE_GATHER, E4B_STAGE_GATE_UP, E4B_STAGE_DOWN, E4B_STAGE_COMBINE = range(5)
 (E4B_WS_TOPK_IDS, E4B_WS_TOPK_W, E4B_WS_EXPERT_OFFSETS, E4B_WS_SORTED_SLOT, E4B_WS_X_SORTED, E4B_WS_H,
  E4B_WS_Y) = range(7)
@@ -36,12 +36,17 @@ class MoeDesc(ctypes.Structure):
         ("E", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32), ("k", ctypes.c_int32),
         ("format", ctypes.c_int32), ("lora_rank", ctypes.c_int32), ("lora_scale", ctypes.c_float),
         ("act", ctypes.c_int32), ("tokens_per_tile", ctypes.c_int32),
+        ("glu_alpha", ctypes.c_float), ("glu_limit", ctypes.c_float), ("glu_beta", ctypes.c_float),
     ]
 
 
-def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0):
+def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0, glu=None):
+    """glu None: SwiGLU; glu = (alpha, limit, beta): the clamped GLU (E4B_ACT_CLAMPED_GLU)."""
     f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
-    return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_SWIGLU, tokens_per_tile)
+    if glu is None:
+        return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_SWIGLU, tokens_per_tile, 0.0, 0.0, 0.0)
+    a, lim, b = glu
+    return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_CLAMPED_GLU, tokens_per_tile, a, lim, b)
 
 
 _LIB = None
@@ -52,14 +57,16 @@ _SIGS = {
     "e4b_nf4_codebook": ([_vp], None),
     "e4b_dequant_mxfp4": ([_vp, _vp, _i64, _vp, _vp], _i32),
     "e4b_quantize_nf4": ([_vp, _i64, _vp, _vp, _vp], _i32),
+    "e4b_deinterleave_rows": ([_vp, _vp, _i32, _i32, _i64, _vp], _i32),
     "e4b_route_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "e4b_route": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "e4b_route_noalloc": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
     "e4b_moe_workspace_bytes": ([ctypes.POINTER(MoeDesc), _i32], _sz),
     "e4b_moe_workspace_region": ([ctypes.POINTER(MoeDesc), _i32, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz)], _i32),
-    "e4b_moe_forward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_moe_forward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                         _sz, _vp], _i32),
     "e4b_moe_forward_stage": ([_i32, ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                               _vp, _sz, _vp], _i32),
+                               _vp, _vp, _vp, _sz, _vp], _i32),
     "e4b_device_status": ([_vp, _vp], _i32),
     "e4b_debug_wait_timeout": ([_u32, _vp, _sz, _vp], _i32),
 }
@@ -131,6 +138,13 @@ def e4b_quantize_nf4(x, n, codes, absmax, stream=None):
     return codes, absmax
 
 
+def e4b_deinterleave_rows(inp, out, E, I, row_bytes, stream=None):
+    _need_cuda(inp, out)
+    _check(lib().e4b_deinterleave_rows(_ptr(inp), _ptr(out), E, I, row_bytes, _stream(stream)),
+           "e4b_deinterleave_rows")
+    return out
+
+
 def e4b_route_workspace_bytes(T, E, k):
     return lib().e4b_route_workspace_bytes(T, E, k)
 
@@ -160,20 +174,22 @@ def e4b_moe_workspace_region(desc, T, region):
     return off.value, nbytes.value
 
 
-def e4b_moe_forward(desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, out, ws,
-                    stream=None):
-    _need_cuda(x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, out, ws)
+def e4b_moe_forward(desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias,
+                    dn_bias, out, ws, stream=None):
+    _need_cuda(x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias, dn_bias, out, ws)
     _check(lib().e4b_moe_forward(ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(gu_codes), _ptr(gu_scales),
-                                 _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B), _ptr(out), _ptr(ws),
-                                 ws.numel() * ws.element_size(), _stream(stream)), "e4b_moe_forward")
+                                 _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B), _ptr(gu_bias),
+                                 _ptr(dn_bias), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream)), "e4b_moe_forward")
     return out
 
 
 def e4b_moe_forward_stage(stage, desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B,
-                          out, ws, stream=None):
+                          gu_bias, dn_bias, out, ws, stream=None):
     _check(lib().e4b_moe_forward_stage(stage, ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(gu_codes),
                                        _ptr(gu_scales), _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B),
-                                       _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+                                       _ptr(gu_bias), _ptr(dn_bias), _ptr(out), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)),
            "e4b_moe_forward_stage")
     return out
 

@@ -37,13 +37,16 @@ def quantize_stack_nf4(w_f32: torch.Tensor, stream=None) -> PackedStack:
 
 class MoeLayer:
     def __init__(self, E, H, I, k, fmt, gate_up: PackedStack, down: PackedStack, lora_A=None, lora_B=None,
-                 lora_scale=0.0, tokens_per_tile=0):
+                 lora_scale=0.0, tokens_per_tile=0, gu_bias=None, dn_bias=None, glu=None):
+        """gu_bias [E, 2I] / dn_bias [E, H] fp32 device tensors (or None) and glu = (alpha, limit, beta)
+        select the gpt-oss epilogue; gate_up rows must already be [gate | up] (see deinterleave_gate_up)."""
         self.E, self.H, self.I, self.k, self.fmt = E, H, I, k, fmt
         self.gate_up, self.down = gate_up, down
         self.lora_A, self.lora_B = lora_A, lora_B
+        self.gu_bias, self.dn_bias = gu_bias, dn_bias
         self.lora_rank = 0 if lora_A is None else lora_A.shape[-1]
         self.lora_scale = lora_scale
-        self.desc = e4b.make_desc(E, H, I, k, fmt, self.lora_rank, lora_scale, tokens_per_tile)
+        self.desc = e4b.make_desc(E, H, I, k, fmt, self.lora_rank, lora_scale, tokens_per_tile, glu)
         self._ws = None
 
     def workspace(self, T, device):
@@ -62,7 +65,8 @@ class MoeLayer:
             out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x_bits.device)
         ws = self.workspace(T, x_bits.device)
         e4b.e4b_moe_forward(self.desc, T, x_bits, logits_bits, self.gate_up.codes, self.gate_up.scales,
-                            self.down.codes, self.down.scales, self.lora_A, self.lora_B, out, ws, stream)
+                            self.down.codes, self.down.scales, self.lora_A, self.lora_B, self.gu_bias, self.dn_bias,
+                            out, ws, stream)
         return out
 
     def region(self, T, which, dtype):
@@ -115,6 +119,23 @@ class HostForward:
         return self.out
 
 
+def deinterleave_gate_up(stack: PackedStack, bias=None, stream=None):
+    """A gate_up stack (and its [E, 2I] bias) released with gate/up rows interleaved, brought to
+    [gate | up] order on the device by the library's row gather.  Returns (stack, bias)."""
+    E, N, K = stack.E, stack.N, stack.K
+    I = N // 2
+    codes = torch.empty_like(stack.codes)
+    scales = torch.empty_like(stack.scales)
+    e4b.e4b_deinterleave_rows(stack.codes, codes, E, I, K // 2, stream)
+    e4b.e4b_deinterleave_rows(stack.scales, scales, E, I, stack.scales.numel() * stack.scales.element_size() // (E * N),
+                              stream)
+    out_bias = None
+    if bias is not None:
+        out_bias = torch.empty_like(bias)
+        e4b.e4b_deinterleave_rows(bias, out_bias, E, I, bias.element_size(), stream)
+    return PackedStack(codes, scales, E, N, K, stack.fmt), out_bias
+
+
 def bits_tensor(bits_np, device):
     """uint16 bf16 bit patterns (NumPy) -> a bf16 device tensor."""
     return torch.from_numpy(np.ascontiguousarray(bits_np).view(np.int16)).to(device).view(torch.bfloat16)
@@ -125,6 +146,9 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
 
     MXFP4 stacks are drawn directly as codes and scales; NF4 stacks are drawn
     as fp32 N(0, std) weights and quantised on the device by the library.
+    With ``w.interleaved`` the drawn gate_up stack (and its bias) is read as a
+    released stack with gate/up rows interleaved and de-interleaved on the
+    device; ``w.bias_std`` and ``w.glu`` select the gpt-oss epilogue.
     """
     E, H, I = w.E, w.H, w.I
     if w.fmt == "mxfp4":
@@ -142,7 +166,13 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
     if w.lora_rank:
         A = bits_tensor(synth.normal_bf16((E, H, w.lora_rank), 1.0 / w.lora_rank, w.seed, "lora_A"), device)
         B = bits_tensor(synth.normal_bf16((E, w.lora_rank, 2 * I), 0.01, w.seed, "lora_B"), device)
-    return MoeLayer(E, H, I, w.k, w.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile)
+    bgu = bdn = None
+    if w.bias_std > 0:
+        bgu = torch.from_numpy(synth.normal_f32((E, 2 * I), w.bias_std, w.seed, "gate_up_bias")).to(device)
+        bdn = torch.from_numpy(synth.normal_f32((E, H), w.bias_std, w.seed, "down_bias")).to(device)
+    if w.interleaved:
+        gu, bgu = deinterleave_gate_up(gu, bgu)
+    return MoeLayer(E, H, I, w.k, w.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu)
 
 
 def synthetic_tokens(w: Workload, T, seed_offset=0):

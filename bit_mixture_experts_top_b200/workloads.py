@@ -23,6 +23,9 @@ class Workload:
     lora_rank: int = 0
     lora_alpha: float = 0.0
     zipf_s: Optional[float] = None        # skewed routing when set
+    glu: Optional[Tuple[float, float, float]] = None   # clamped GLU (alpha, limit, beta); None = SwiGLU
+    bias_std: float = 0.0                 # > 0: per-expert fp32 biases N(0, bias_std) on both stacks
+    interleaved: bool = False             # gate_up drawn with gate/up rows interleaved, de-interleaved at load
     seed: int = 0
     notes: str = field(default="", compare=False)
 

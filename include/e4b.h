@@ -22,6 +22,9 @@
  *         per 64 NF4 weights; the stock expert epilogue act(gate)*up with no
  *         biases or clamps; "Current measured position": routing is decided
  *         on the router logits.
+ *   [MX] "Why it happens" also names what gpt-oss adds to that epilogue:
+ *         per-expert biases, interleaved gate/up rows and a clamped GLU;
+ *         "Which project solves it": its module de-interleaves the rows.
  *
  * Conventions for every entry point:
  *   - Device pointers are plain CUDA device addresses; the caller owns every
@@ -40,8 +43,10 @@
  * Storage layouts (readings of the pages where they are silent):
  *   - Expert stacks are stored K-contiguous: gate_up as [E, 2I, H] (logical
  *     [E, H, 2I] transposed), down as [E, H, I]; the fused 2I rows are
- *     [gate rows 0..I-1 | up rows I..2I-1].  Quantisation blocks are runs of
- *     the flat stored stack, hence along K.
+ *     [gate rows 0..I-1 | up rows I..2I-1] (a stack released with gate/up
+ *     rows interleaved is brought to this order once, by
+ *     e4b_deinterleave_rows).  Quantisation blocks are runs of the flat
+ *     stored stack, hence along K.
  *   - MXFP4: element 2j is the LOW nibble of byte j; scale byte b covers
  *     elements [32b, 32b+32); value = e2m1(code) * 2^(scale - 127), 0xFF = NaN.
  *   - NF4: element 2j is the HIGH nibble of byte j; absmax[b] (fp32) covers
@@ -57,7 +62,7 @@
 extern "C" {
 #endif
 
-#define E4B_ABI_VERSION 1
+#define E4B_ABI_VERSION 2
 
 typedef enum {
   E4B_OK = 0,
@@ -68,7 +73,13 @@ typedef enum {
 } e4b_status;
 
 enum { E4B_NF4 = 0, E4B_MXFP4 = 1 };   /* e4b_moe_desc.format */
-enum { E4B_ACT_SWIGLU = 0 };           /* e4b_moe_desc.act: h = silu(gate) * up */
+/* e4b_moe_desc.act.  E4B_ACT_SWIGLU: h = silu(gate) * up, silu(z) = z / (1 + e^-z).
+ * E4B_ACT_CLAMPED_GLU (gpt-oss, [MX] "Why it happens"; the pages give no formula or
+ * constants, so this is the library's reading, with the constants as parameters):
+ *   g = min(gate, glu_limit), u = clamp(up, -glu_limit, glu_limit),
+ *   h = g * sigmoid(glu_alpha * g) * (u + glu_beta).
+ * The public gpt-oss release uses glu_alpha = 1.702, glu_limit = 7, glu_beta = 1. */
+enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 };
 
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st* e4b_stream;
@@ -82,13 +93,16 @@ typedef struct {
   int32_t format;          /* E4B_NF4 or E4B_MXFP4 */
   int32_t lora_rank;       /* 0 = no LoRA; else 1..16 */
   float lora_scale;        /* alpha / r, multiplies the LoRA delta */
-  int32_t act;             /* E4B_ACT_SWIGLU */
+  int32_t act;             /* E4B_ACT_SWIGLU or E4B_ACT_CLAMPED_GLU */
   int32_t tokens_per_tile; /* 0 = chosen by the library (the decode kernel when the mean number of rows
                               per routed expert is at most 12, else a tcgen05 tile); 8 = decode kernel
                               (codes decoded in registers, warp-level MMA; tokens go in chunks of 8, 16
                               or 32 by the mean rows per expert; needs the scale rows of 128 weight rows
                               of both stacks to fit in shared memory, else E4B_ERR_UNSUPPORTED);
                               32, 64, 128, 192 or 256 = tcgen05 tile width */
+  float glu_alpha;         /* E4B_ACT_CLAMPED_GLU only: finite */
+  float glu_limit;         /* E4B_ACT_CLAMPED_GLU only: > 0, +inf allowed (no clamp) */
+  float glu_beta;          /* E4B_ACT_CLAMPED_GLU only: finite */
 } e4b_moe_desc;
 
 /* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */
@@ -128,6 +142,22 @@ e4b_status e4b_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_
  */
 e4b_status e4b_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax,
                             e4b_stream stream);
+
+/*
+ * gpt-oss gate_up de-interleave (load-time layout step).  [MX] "Why it
+ * happens" (interleaved gate/up rows), "Which project solves it" (the gpt-oss
+ * module de-interleaves them).
+ *   in        : [E, 2I] rows of row_bytes bytes each, gate i at row 2i and
+ *               up i at row 2i + 1                      (device, read)
+ *   out       : [E, 2I] rows, gate rows 0..I-1 then up rows I..2I-1 (device,
+ *               written); must not overlap `in`
+ *   row_bytes : bytes per row, >= 0 (H/2 for packed codes, the scale bytes of
+ *               one row, 4 for one fp32 bias per row)
+ * A pure byte permutation: exact.  Any alignment is accepted (16- and 4-byte
+ * aligned rows move in wider words).
+ */
+e4b_status e4b_deinterleave_rows(const void* in, void* out, int32_t E, int32_t I, int64_t row_bytes,
+                                 e4b_stream stream);
 
 /* Workspace bytes e4b_route needs for T tokens, E experts, k choices. */
 size_t e4b_route_workspace_bytes(int32_t T, int32_t E, int32_t k);
@@ -181,7 +211,8 @@ size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
 /*
  * Layer forward.  [IX] grouped gate_up GEMM with in-kernel dequant, optional
  * per-expert LoRA delta before the activation, [PKG] SwiGLU epilogue
- * act(gate)*up, grouped down GEMM, then the weighted combine
+ * act(gate)*up (or [MX] the gpt-oss biases and clamped GLU, per d->act and
+ * the bias pointers), grouped down GEMM, then the weighted combine
  * out[t] = sum_j w[t,j] * y[t,j] in fp32, j ascending, rounded to bf16.
  *   x         : [T, H] bf16                            (device, read)
  *   logits    : [T, E] bf16                            (device, read)
@@ -190,6 +221,10 @@ size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
  *   dn_codes  : [E, H, I] packed 4-bit;  dn_scales as gu_scales for [E, H, I]
  *   lora_A    : [E, H, r] bf16 or NULL;  lora_B : [E, r, 2I] bf16 or NULL
  *               (both or neither, and r == d->lora_rank)
+ *   gu_bias   : [E, 2I] fp32 as [gate | up], or NULL (no bias); added to
+ *               the gate_up output before the activation
+ *   dn_bias   : [E, H] fp32 or NULL; added to each expert's down output, so
+ *               the combine weights scale it too
  *   out       : [T, H] bf16                            (device, written)
  *   ws        : workspace, 256-byte aligned, >= e4b_moe_workspace_bytes(d, T);
  *               its first 256 bytes hold the device status word and the decode
@@ -201,15 +236,16 @@ size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
 e4b_status e4b_moe_forward(const e4b_moe_desc* d, int32_t T, const uint16_t* x,
                            const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
                            const uint8_t* dn_codes, const void* dn_scales,
-                           const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* out,
+                           const uint16_t* lora_A, const uint16_t* lora_B,
+                           const float* gu_bias, const float* dn_bias, uint16_t* out,
                            void* ws, size_t ws_bytes, e4b_stream stream);
 
 /* Stages of e4b_moe_forward, in order. */
 enum {
   E4B_STAGE_ROUTE = 0,     /* clears the status word; top-k, histogram, stable permute */
   E4B_STAGE_GATHER = 1,    /* routed rows in expert order (+ LoRA left factor x.A_e) */
-  E4B_STAGE_GATE_UP = 2,   /* grouped gate_up GEMM with dequant, LoRA delta, SwiGLU -> h */
-  E4B_STAGE_DOWN = 3,      /* grouped down GEMM with dequant -> y */
+  E4B_STAGE_GATE_UP = 2,   /* grouped gate_up GEMM with dequant, LoRA delta, bias, activation -> h */
+  E4B_STAGE_DOWN = 3,      /* grouped down GEMM with dequant (+ bias) -> y */
   E4B_STAGE_COMBINE = 4    /* out[t] = sum_j w[t,j] * y[t,j] */
 };
 
@@ -222,7 +258,8 @@ enum {
 e4b_status e4b_moe_forward_stage(int32_t stage, const e4b_moe_desc* d, int32_t T, const uint16_t* x,
                                  const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
                                  const uint8_t* dn_codes, const void* dn_scales,
-                                 const uint16_t* lora_A, const uint16_t* lora_B, uint16_t* out,
+                                 const uint16_t* lora_A, const uint16_t* lora_B,
+                                 const float* gu_bias, const float* dn_bias, uint16_t* out,
                                  void* ws, size_t ws_bytes, e4b_stream stream);
 
 /* Intermediate buffers inside a forward workspace, for inspection. */
@@ -232,7 +269,7 @@ enum {
   E4B_WS_EXPERT_OFFSETS = 2, /* int32 [E+1] */
   E4B_WS_SORTED_SLOT = 3,  /* int32 [T*k] */
   E4B_WS_X_SORTED = 4,     /* bf16  [T*k, H] */
-  E4B_WS_H = 5,            /* bf16  [T*k, I]  silu(gate)*up per routed row */
+  E4B_WS_H = 5,            /* bf16  [T*k, I]  act(gate, up) per routed row */
   E4B_WS_Y = 6             /* fp32  [T*k, H]  down output per routed row */
 };
 

@@ -91,6 +91,17 @@ def oracle_lora(w):
     return A, B
 
 
+def oracle_epilogue(w):
+    """(gate_up bias, down bias) of the workload as the oracle sees them (de-interleaved when released so)."""
+    if w.bias_std <= 0:
+        return None, None
+    bgu = synth.normal_f32((w.E, 2 * w.I), w.bias_std, w.seed, "gate_up_bias")
+    bdn = synth.normal_f32((w.E, w.H), w.bias_std, w.seed, "down_bias")
+    if w.interleaved:
+        bgu = omoe.deinterleave_rows(bgu, w.E, w.I)
+    return bgu, bdn
+
+
 def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=0, x=None, logits=None):
     """Runs the GPU forward on all T tokens and compares `sample` rows (default all) with the oracle."""
     dev = device()
@@ -104,10 +115,15 @@ def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=
     rows = np.arange(T) if sample is None else np.asarray(sample)
     experts = touched_experts(logits[rows], w.k)
     ref_stacks = oracle_stacks(w, experts)
+    if w.interleaved:
+        gc, gs, dc, ds = ref_stacks
+        ref_stacks = (omoe.deinterleave_rows(gc, w.E, w.I), omoe.deinterleave_rows(gs, w.E, w.I), dc, ds)
     if w.fmt == "nf4":
         check_nf4_stacks_equal(lay, w, experts, ref_stacks)
     A, B = oracle_lora(w)
+    bgu, bdn = oracle_epilogue(w)
     ref, _ = omoe.moe_forward(x[rows], logits[rows], w.k, w.fmt, w.E, w.H, w.I, *ref_stacks,
-                              lora_A_bits=A, lora_B_bits=B, lora_scale=w.lora_scale)
+                              lora_A_bits=A, lora_B_bits=B, lora_scale=w.lora_scale, gu_bias=bgu, dn_bias=bdn,
+                              glu=w.glu)
     got = bf16_to_f64(out)[rows]
     return assert_close_layer(got, ref, f"{w.name} T={T} tile={tokens_per_tile}"), lay, out

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_function(L):
 
 
 def test_abi_version(L):
-    assert e4b.e4b_abi_version() == 1
+    assert e4b.e4b_abi_version() == 2
     assert L.e4b_status_string(4).decode().startswith("E4B_ERR_TIMEOUT")
 
 
@@ -63,19 +63,34 @@ def test_forward_validation_and_workspace(L):
                 e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=17),
                 e4b.make_desc(8, 256, 128, 2, "nf4", tokens_per_tile=48),
                 # decode kernel asked for, but 128 rows of 8192/64 fp32 scales per unit do not fit
-                e4b.make_desc(8, 8192, 128, 2, "nf4", tokens_per_tile=8)]:
+                e4b.make_desc(8, 8192, 128, 2, "nf4", tokens_per_tile=8),
+                # clamped GLU needs a positive limit and finite alpha / beta
+                e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(1.702, 0.0, 1.0)),
+                e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(float("nan"), 7.0, 1.0)),
+                e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(1.702, 7.0, float("inf")))]:
         assert e4b.e4b_moe_workspace_bytes(bad, 64) == 0
     # the same shape is served by the tcgen05 tiles, and by the decode kernel at 2048
     assert e4b.e4b_moe_workspace_bytes(e4b.make_desc(8, 8192, 128, 2, "nf4"), 64) > 0
     assert e4b.e4b_moe_workspace_bytes(e4b.make_desc(8, 2048, 128, 2, "nf4", tokens_per_tile=8), 64) > 0
     # one-sided LoRA is refused before any launch
     dl = e4b.make_desc(8, 256, 128, 2, "nf4", lora_rank=8, lora_scale=2.0)
-    st = L.e4b_moe_forward(ctypes.byref(dl), 4, None, None, None, None, None, None, 256, None, None, 256,
-                           1 << 30, None)
+    st = L.e4b_moe_forward(ctypes.byref(dl), 4, None, None, None, None, None, None, 256, None, None, None, None,
+                           256, 1 << 30, None)
     assert st == e4b.E4B_ERR_INVALID_ARG
     # workspace too small
-    st = L.e4b_moe_forward(ctypes.byref(d), 64, 256, 256, 256, 256, 256, 256, None, None, 256, 256, 1024, None)
+    st = L.e4b_moe_forward(ctypes.byref(d), 64, 256, 256, 256, 256, 256, 256, None, None, None, None, 256, 256, 1024,
+                           None)
     assert st == e4b.E4B_ERR_INVALID_ARG
     off, nb = e4b.e4b_moe_workspace_region(d, 64, e4b.E4B_WS_H)
     assert off % 256 == 0 and nb == 64 * 2 * 128 * 2 and off + nb <= ws
     assert L.e4b_debug_wait_timeout(2_000_000_000, 256, 4096, None) == e4b.E4B_ERR_INVALID_ARG
+
+
+def test_deinterleave_validation(L):
+    # sizes and overlap are checked on the host; empty inputs are a no-op (nothing launched)
+    assert L.e4b_deinterleave_rows(None, None, 0, 64, 1440, None) == e4b.E4B_OK
+    assert L.e4b_deinterleave_rows(None, None, 4, 64, 0, None) == e4b.E4B_OK
+    assert L.e4b_deinterleave_rows(256, 512, -1, 64, 16, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_deinterleave_rows(None, 512, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_deinterleave_rows(256, 256 + 16, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG   # overlap
+    assert L.e4b_deinterleave_rows(256 + 16, 256, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG

@@ -1,6 +1,7 @@
 """GPU parity of the full layer forward (route -> grouped gate_up with dequant,
-LoRA, SwiGLU -> grouped down -> combine) against the fp64 oracle, within
-relative Frobenius 5e-3 and max-abs 3e-2 * max|ref|."""
+LoRA, SwiGLU or the gpt-oss biases and clamped GLU -> grouped down -> combine)
+against the fp64 oracle, within relative Frobenius 5e-3 and max-abs
+3e-2 * max|ref|."""
 import numpy as np
 import pytest
 import torch
@@ -114,6 +115,57 @@ def test_gptoss_20b_prefill_sampled():
 
 def test_gptoss_120b_zipf_prefill_sampled():
     run_and_compare(OSS120, 16384, sample=np.random.default_rng(2).choice(16384, 24, replace=False))
+
+
+# ---------------------------------------------------------------- gpt-oss epilogue
+
+GLU = (1.702, 7.0, 1.0)     # alpha, limit, up offset of the public gpt-oss release
+
+
+@pytest.mark.parametrize("tpt", [0, 8, 64, 256])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nf4"])
+def test_gptoss_epilogue_small(fmt, tpt):
+    # biases on both stacks, clamped GLU, gate/up rows released interleaved and de-interleaved on the
+    # device; the limits clamp about a fifth of the gate values and half of the up values
+    glu = GLU if fmt == "mxfp4" else (1.702, 0.5, 1.0)
+    w = Workload(f"oss_{fmt}", fmt, E=6, H=320, I=192, k=2, tokens=(100,), exp_range=(-6, -1), glu=glu,
+                 bias_std=0.5, interleaved=True, seed=21)
+    run_and_compare(w, 100, tokens_per_tile=tpt)
+
+
+@pytest.mark.parametrize("tpt", [0, 256])
+def test_gptoss_20b_epilogue_decode(tpt):
+    w = Workload("oss20_glu", "mxfp4", E=32, H=2880, I=2880, k=4, tokens=(16,), exp_range=(-6, 1), glu=GLU,
+                 bias_std=0.5, interleaved=True)
+    run_and_compare(w, 16, tokens_per_tile=tpt)
+
+
+@pytest.mark.parametrize("tpt", [0, 8, 128])
+def test_unclamped_glu_with_zero_bias_is_swiglu(tpt):
+    # alpha 1, no clamp, no up offset, zero biases: the stock epilogue's values (zeros may differ in sign)
+    dev = device()
+    lay = layer.synthetic_layer(TINY, dev, tpt)
+    x, logits = layer.synthetic_tokens(TINY, 64)
+    xb, lb = layer.bits_tensor(x, dev), layer.bits_tensor(logits, dev)
+    base = lay.forward(xb, lb).clone()
+    z_gu = torch.zeros((TINY.E, 2 * TINY.I), dtype=torch.float32, device=dev)
+    z_dn = torch.zeros((TINY.E, TINY.H), dtype=torch.float32, device=dev)
+    glu = layer.MoeLayer(TINY.E, TINY.H, TINY.I, TINY.k, TINY.fmt, lay.gate_up, lay.down, tokens_per_tile=tpt,
+                         gu_bias=z_gu, dn_bias=z_dn, glu=(1.0, float("inf"), 0.0))
+    assert torch.equal(glu.forward(xb, lb).float(), base.float())
+
+
+@pytest.mark.parametrize("row_bytes,offset", [(1440, 0), (90, 0), (4, 0), (16, 0), (64, 1)])
+def test_deinterleave_rows_bit_exact(row_bytes, offset):
+    from oracle import moe as omoe
+    E, I = 3, 37
+    a = np.random.default_rng(row_bytes).integers(0, 256, size=E * 2 * I * row_bytes, dtype=np.uint8)
+    dev = device()
+    buf = torch.zeros(a.size + 16, dtype=torch.uint8, device=dev)
+    buf[offset:offset + a.size] = torch.from_numpy(a).to(dev)
+    out = torch.full((a.size,), 0xAB, dtype=torch.uint8, device=dev)
+    e4b.e4b_deinterleave_rows(buf[offset:offset + a.size], out, E, I, row_bytes)
+    assert np.array_equal(out.cpu().numpy(), omoe.deinterleave_rows(a, E, I))
 
 
 def test_forward_is_deterministic_and_permutation_consistent():
