@@ -98,16 +98,17 @@ def deinterleave_rows(stack, E, I):
 
 
 def moe_forward(x_bits, logits_bits, k, fmt, E, H, I, gu_codes, gu_scales, dn_codes, dn_scales,
-                lora_A_bits=None, lora_B_bits=None, lora_scale=0.0, gu_bias=None, dn_bias=None, glu=None):
+                lora_A_bits=None, lora_B_bits=None, lora_scale=0.0, gu_bias=None, dn_bias=None, glu=None,
+                gating="topk"):
     """Layer forward.  x: bf16 bits [T, H]; logits: bf16 bits [T, E].  Returns (out fp64 [T, H], route dict).
 
     gu_bias [E, 2I] / dn_bias [E, H] (fp32, or None for no bias) and
     glu = (alpha, limit, beta) select the gpt-oss epilogue; glu None is the
-    stock SwiGLU silu(gate) * up.
+    stock SwiGLU silu(gate) * up.  gating selects the router weights (:func:`oracle.route.route`).
     """
     x = bf16_bits_to_f64(np.asarray(x_bits, dtype=np.uint16)).reshape(-1, H)
     T = x.shape[0]
-    r = route(np.asarray(logits_bits, dtype=np.uint16).reshape(T, E), k)
+    r = route(np.asarray(logits_bits, dtype=np.uint16).reshape(T, E), k, gating)
     offsets, sorted_slot = r["offsets"], r["sorted_slot"]
     x_sorted = x[sorted_slot // k]                       # step 2: permute
     y_sorted = np.zeros((T * k, H), dtype=np.float64)

@@ -20,7 +20,9 @@ Readings where the pages are silent:
   +0.  NaN logits are outside the contract.
 * The gate weights are the softmax over the k selected logits (equivalently a
   softmax over all E followed by renormalisation of the top k), computed in
-  fp64 and stored in fp32.
+  fp64 and stored in fp32.  The other gating of the named families (a softmax
+  over all E whose top k are kept without renormalising, so they sum to less
+  than 1) is the ``gating="all"`` option.
 * Slot s = t*k + j is token t's j-th choice.  ``expert_offsets`` is the
   exclusive prefix sum of the per-expert slot counts; ``sorted_slot`` lists
   the slots grouped by expert id, each group in ascending slot order (a stable
@@ -47,6 +49,13 @@ def softmax_selected(logits, ids):
     return ez / ez.sum(axis=1, keepdims=True)
 
 
+def softmax_all_selected(logits, ids):
+    """fp64 softmax over all E logits of each token, read at the selected ids (not renormalised)."""
+    z = logits - logits.max(axis=1, keepdims=True)
+    ez = np.exp(z)
+    return np.take_along_axis(ez, ids.astype(np.int64), axis=1) / ez.sum(axis=1, keepdims=True)
+
+
 def permute(ids, E):
     """Histogram, exclusive offsets, stable expert-grouped slot order and its inverse."""
     flat = ids.reshape(-1).astype(np.int64)
@@ -59,13 +68,17 @@ def permute(ids, E):
     return counts.astype(np.int32), offsets.astype(np.int32), sorted_slot, slot_pos
 
 
-def route(logits_bits, k):
-    """bf16 logits bit patterns [T, E] -> dict of ids, weights (fp64 and fp32), counts, offsets, permutation."""
+def route(logits_bits, k, gating="topk"):
+    """bf16 logits bit patterns [T, E] -> dict of ids, weights (fp64 and fp32), counts, offsets, permutation.
+
+    gating "topk": softmax over the k selected logits; "all": softmax over all E, top k kept as they are.
+    """
     logits = bf16_bits_to_f64(np.asarray(logits_bits, dtype=np.uint16))
     T, E = logits.shape
-    assert 1 <= k <= E
+    assert 1 <= k <= E and gating in ("topk", "all")
     ids = topk_select(logits, k) if T else np.zeros((0, k), np.int32)
-    w = softmax_selected(logits, ids) if T else np.zeros((0, k))
+    gate = softmax_selected if gating == "topk" else softmax_all_selected
+    w = gate(logits, ids) if T else np.zeros((0, k))
     counts, offsets, sorted_slot, slot_pos = permute(ids, E)
     return {
         "ids": ids,

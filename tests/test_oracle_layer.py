@@ -51,6 +51,30 @@ def test_route_weights_equal_renormalised_full_softmax():
     assert np.all(np.diff(r["w64"], axis=1) <= 0)          # ordered by logit
 
 
+def test_route_full_softmax_gating_is_unrenormalised_top_k():
+    import scipy.special
+    g = np.random.default_rng(16)
+    logits = synth.to_bf16_bits(g.standard_normal((64, 32)) * 2)
+    lf = bf16.bf16_bits_to_f64(logits)
+    for k in (1, 4, 32):
+        ra, rt = route.route(logits, k, "all"), route.route(logits, k)
+        assert np.array_equal(ra["ids"], rt["ids"])
+        full = scipy.special.softmax(lf, axis=1)
+        assert np.allclose(ra["w64"], np.take_along_axis(full, ra["ids"].astype(np.int64), 1), rtol=1e-13, atol=0)
+        s = ra["w64"].sum(axis=1)
+        assert np.all(s <= 1 + 1e-15) and (k < 32 or np.allclose(s, 1.0, rtol=1e-14, atol=0))
+        assert np.allclose(ra["w64"] / s[:, None], rt["w64"], rtol=1e-13, atol=0)   # renormalising gives top-k
+    # the forward takes whichever weights the router gives
+    E, H, I, k, T = 4, 64, 64, 2, 6
+    gu, dn = _tiny_layer("mxfp4", E, H, I, seed=16)
+    x = synth.normal_bf16((T, H), 1.0, 16, "x")
+    lg = synth.normal_bf16((T, E), 1.0, 16, "logits")
+    out_t, r_t = moe.moe_forward(x, lg, k, "mxfp4", E, H, I, gu[0], gu[1], dn[0], dn[1])
+    out_a, r_a = moe.moe_forward(x, lg, k, "mxfp4", E, H, I, gu[0], gu[1], dn[0], dn[1], gating="all")
+    scale = r_a["w64"].sum(axis=1, keepdims=True)        # per-token mass of the kept experts
+    assert np.allclose(out_a, out_t * scale, rtol=1e-12, atol=1e-12 * np.abs(out_t).max())
+
+
 def test_route_permutation_is_stable_grouping():
     g = np.random.default_rng(6)
     T, E, k = 300, 16, 3
