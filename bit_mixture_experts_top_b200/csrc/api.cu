@@ -97,6 +97,7 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
       (!std::isfinite(d->glu_alpha) || !std::isfinite(d->glu_beta) || !(d->glu_limit > 0.0f)))
     return E4B_ERR_INVALID_ARG;
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
+  if (d->gating != E4B_GATE_SOFTMAX_TOPK && d->gating != E4B_GATE_SOFTMAX_ALL) return E4B_ERR_INVALID_ARG;
   const int tpt = d->tokens_per_tile;
   if (tpt == 8 && !(skinny_gemm_supported(d->H, d->format) && skinny_gemm_supported(d->I, d->format)))
     return E4B_ERR_UNSUPPORTED;
@@ -201,10 +202,12 @@ size_t e4b_route_workspace_bytes(int32_t T, int32_t E, int32_t k) {
   return route_layout(T, E, k).total;
 }
 
-e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
+e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating, int32_t* topk_ids,
+                     float* topk_w,
                      int32_t* expert_offsets, int32_t* sorted_slot, void* ws, size_t ws_bytes,
                      e4b_stream stream) {
   if (T < 0 || E < 1 || k < 1 || k > E) return E4B_ERR_INVALID_ARG;
+  if (gating != E4B_GATE_SOFTMAX_TOPK && gating != E4B_GATE_SOFTMAX_ALL) return E4B_ERR_INVALID_ARG;
   if (E > kMaxExperts || k > kMaxTopK) return E4B_ERR_UNSUPPORTED;
   if (!expert_offsets || !ws || !aligned(ws, kAlign)) return E4B_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !topk_ids || !topk_w || !sorted_slot)) return E4B_ERR_INVALID_ARG;
@@ -223,7 +226,7 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, in
   b.sorted_slot = sorted_slot;
   b.slot_pos = at<int32_t>(ws, L.slot_pos);
   // the status words are zeroed by the launch sequence (in-kernel for one routing block)
-  return launch_route(logits, T, E, k, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  return launch_route(logits, T, E, k, gating, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }
 
 size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T) {
@@ -312,7 +315,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
     switch (stage) {
       case E4B_STAGE_ROUTE:
         // zeroes the status words first (in the routing kernel when one block routes)
-        if (launch_route(logits, T, d->E, d->k, tpt, b, b.status, s) != cudaSuccess) return E4B_ERR_CUDA;
+        if (launch_route(logits, T, d->E, d->k, d->gating, tpt, b, b.status, s) != cudaSuccess) return E4B_ERR_CUDA;
         break;
       case E4B_STAGE_GATHER:
         if (launch_gather(x, d->H, d->k, R, b.sorted_slot, b.topk_ids, d->E, x_sorted, lora_A, d->lora_rank,

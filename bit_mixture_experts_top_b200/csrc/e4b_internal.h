@@ -49,7 +49,8 @@ inline int route_blocks(int32_t T) { return (T + kRouteTokensPerBlock - 1) / kRo
 // Routing kernels.  status_words (kStatusBytes, or null) are zeroed before
 // anything else runs: inside the single routing block for T <= 128, else by a
 // memset ahead of the multi-block kernels.
-cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t tokens_per_tile,
+cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
+                         int32_t tokens_per_tile,
                          const RouteBuffers& b, int32_t* status_words, cudaStream_t s);
 
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n, uint16_t* out,

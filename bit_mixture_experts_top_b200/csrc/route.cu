@@ -9,7 +9,10 @@
 //     packed into 32-bit keys (order-preserving bf16 bits << 16 | 0xFFFF - id),
 //     so one unsigned max picks the largest logit and, on ties, the lowest id;
 //     k rounds of __reduce_max_sync select the k experts;
-//   * gate weights are the fp32 softmax of the k selected logits;
+//   * gate weights are the fp32 softmax of the k selected logits, or (gating
+//     E4B_GATE_SOFTMAX_ALL) the softmax over all E logits read at the k picks,
+//     not renormalised: the denominator is summed from the keys before the
+//     first pick is removed;
 //   * the block histogram feeds per-block counts; the last block to finish
 //     turns them into expert offsets, per-block bases and tile-chunk offsets;
 //   * the rank kernel orders each block's slots by (expert, slot) with
@@ -38,6 +41,24 @@ __device__ __forceinline__ uint32_t route_key(uint16_t bits, int e) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+// The logit a key holds (inverse of route_key's order-preserving map).
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  const uint32_t ord = key >> 16;
+  return bf16_bits_to_f32(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu)));
+}
+
+// sum over the row of exp(logit - m), from this warp's keys (0 = no expert)
+template <int J>
+__device__ __forceinline__ float row_exp_sum(const uint32_t (&key)[J], float m) {
+  float s = 0.0f;
+#pragma unroll
+  for (int j = 0; j < J; ++j)
+    if (key[j]) s += expf(key_logit(key[j]) - m);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
+  return s;
+}
 
 // Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
 // slots of the block with the same expert).  Each warp owns a contiguous
@@ -94,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __r
 }
 
 __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E,
-                                                                  int k, int tokens_per_tile, int nblk,
+                                                                  int k, int gating, int tokens_per_tile, int nblk,
                                                                   int32_t* __restrict__ topk_ids,
                                                                   float* __restrict__ topk_w, int32_t* block_counts,
                                                                   uint32_t* done_counter, int32_t* expert_offsets,
@@ -127,11 +148,13 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
     const int t = t_begin + warp + kTopkWarps * q;
     if (t >= T) break;
     uint32_t mine = 0;                     // lane j keeps the j-th pick
+    float all_sum = 0.0f;                  // full-softmax denominator (E4B_GATE_SOFTMAX_ALL)
     for (int r = 0; r < k; ++r) {
       uint32_t best = 0;
 #pragma unroll
       for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
       best = __reduce_max_sync(kFull, best);
+      if (r == 0 && gating == E4B_GATE_SOFTMAX_ALL) all_sum = row_exp_sum(key[q], key_logit(best));
       const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
 #pragma unroll
       for (int j = 0; j < kMaxExperts / 32; ++j)
@@ -142,8 +165,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
     float v = 0.0f;
     if (lane < k) {
       id = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
-      const uint32_t ord = mine >> 16;     // invert route_key: the bf16 bits of the pick
-      v = bf16_bits_to_f32(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu)));
+      v = key_logit(mine);
     }
     const float m = __shfl_sync(kFull, v, 0);          // the first pick holds the maximum
     float ex = (lane < k) ? expf(v - m) : 0.0f;
@@ -152,7 +174,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
     if (lane < k) {
       topk_ids[static_cast<int64_t>(t) * k + lane] = id;
-      topk_w[static_cast<int64_t>(t) * k + lane] = ex / sum;
+      topk_w[static_cast<int64_t>(t) * k + lane] = ex / (gating == E4B_GATE_SOFTMAX_ALL ? all_sum : sum);
       atomicAdd(&s_cnt[id], 1);
     }
   }
@@ -232,7 +254,8 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
 // The block also zeroes the status words of the workspace first (the caller
 // skips its memset), so a small forward starts with a single launch.
 __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
-                                                                  int k, int tokens_per_tile, int32_t* status_words,
+                                                                  int k, int gating, int tokens_per_tile,
+                                                                  int32_t* status_words,
                                                                   int32_t* __restrict__ topk_ids,
                                                                   float* __restrict__ topk_w,
                                                                   int32_t* __restrict__ expert_offsets,
@@ -266,11 +289,13 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
     const int t = warp + kTopkWarps * q;
     if (t >= T) break;
     uint32_t mine = 0;
+    float all_sum = 0.0f;
     for (int r = 0; r < k; ++r) {
       uint32_t best = 0;
 #pragma unroll
       for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
       best = __reduce_max_sync(kFull, best);
+      if (r == 0 && gating == E4B_GATE_SOFTMAX_ALL) all_sum = row_exp_sum(key[q], key_logit(best));
       const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
 #pragma unroll
       for (int j = 0; j < kMaxExperts / 32; ++j)
@@ -281,8 +306,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
     float v = 0.0f;
     if (lane < k) {
       id = 0xFFFF - static_cast<int>(mine & 0xFFFFu);
-      const uint32_t ord = mine >> 16;
-      v = bf16_bits_to_f32(static_cast<uint16_t>((ord & 0x8000u) ? (ord & 0x7FFFu) : (~ord & 0xFFFFu)));
+      v = key_logit(mine);
     }
     const float m = __shfl_sync(kFull, v, 0);
     float ex = (lane < k) ? expf(v - m) : 0.0f;
@@ -291,7 +315,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
     if (lane < k) {
       topk_ids[static_cast<int64_t>(t) * k + lane] = id;
-      topk_w[static_cast<int64_t>(t) * k + lane] = ex / sum;
+      topk_w[static_cast<int64_t>(t) * k + lane] = ex / (gating == E4B_GATE_SOFTMAX_ALL ? all_sum : sum);
       s_ids[t * k + lane] = static_cast<int16_t>(id);
       atomicAdd(&s_cnt[id], 1);
     }
@@ -489,7 +513,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
 
 }  // namespace
 
-cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t tokens_per_tile,
+cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
+                         int32_t tokens_per_tile,
                          const RouteBuffers& b, int32_t* status_words, cudaStream_t s) {
   if (T == 0) {
     cudaError_t err = status_words ? cudaMemsetAsync(status_words, 0, kStatusBytes, s) : cudaSuccess;
@@ -499,13 +524,13 @@ cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k
   }
   const int nblk = route_blocks(T);
   if (nblk == 1) {
-    route_small_kernel<<<1, kTopkThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, status_words, b.topk_ids,
+    route_small_kernel<<<1, kTopkThreads, 0, s>>>(logits, T, E, k, gating, tokens_per_tile, status_words, b.topk_ids,
                                                   b.topk_w, b.expert_offsets, b.chunk_off, b.sorted_slot,
                                                   b.slot_pos);
     return cudaGetLastError();
   }
   if (status_words && cudaMemsetAsync(status_words, 0, kStatusBytes, s) != cudaSuccess) return cudaGetLastError();
-  route_topk_kernel<<<nblk, kTopkThreads, 0, s>>>(logits, T, E, k, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
+  route_topk_kernel<<<nblk, kTopkThreads, 0, s>>>(logits, T, E, k, gating, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
                                                b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off,
                                                b.sorted_slot, b.slot_pos);
   cudaError_t err = cudaGetLastError();
@@ -576,11 +601,12 @@ e4b_status route_scratch_address(uint8_t** out) {
 }  // namespace
 }  // namespace e4b
 
-extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_ids,
-                                        float* topk_w, int32_t* expert_offsets, int32_t* sorted_slot,
-                                        e4b_stream stream) {
+extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
+                                        int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
+                                        int32_t* sorted_slot, e4b_stream stream) {
   using namespace e4b;
   if (T < 0 || E < 1 || k < 1 || k > E) return E4B_ERR_INVALID_ARG;
+  if (gating != E4B_GATE_SOFTMAX_TOPK && gating != E4B_GATE_SOFTMAX_ALL) return E4B_ERR_INVALID_ARG;
   if (E > kMaxExperts || k > kMaxTopK) return E4B_ERR_UNSUPPORTED;
   if (!expert_offsets) return E4B_ERR_INVALID_ARG;
   if (T > 0 && (!logits || !topk_ids || !topk_w || !sorted_slot)) return E4B_ERR_INVALID_ARG;
@@ -607,5 +633,5 @@ extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32
   b.block_counts = reinterpret_cast<int32_t*>(scratch + off_counts);
   b.sorted_slot = sorted_slot;
   b.slot_pos = reinterpret_cast<int32_t*>(scratch + off_pos);
-  return launch_route(logits, T, E, k, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  return launch_route(logits, T, E, k, gating, 0, b, b.status, s) == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
 }

@@ -19,6 +19,8 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "e4b.h")
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_UNSUPPORTED, E4B_ERR_CUDA, E4B_ERR_TIMEOUT = range(5)
 E4B_NF4, E4B_MXFP4 = 0, 1
 E4B_ACT_SWIGLU, E4B_ACT_CLAMPED_GLU = 0, 1
+E4B_GATE_SOFTMAX_TOPK, E4B_GATE_SOFTMAX_ALL = 0, 1
+GATINGS = {"topk": E4B_GATE_SOFTMAX_TOPK, "all": E4B_GATE_SOFTMAX_ALL}
 E4B_STAGE_ROUTE, E4B_STAGE_GATHER, E4B_STAGE_GATE_UP, E4B_STAGE_DOWN, E4B_STAGE_COMBINE = range(5)
 (E4B_WS_TOPK_IDS, E4B_WS_TOPK_W, E4B_WS_EXPERT_OFFSETS, E4B_WS_SORTED_SLOT, E4B_WS_X_SORTED, E4B_WS_H,
  E4B_WS_Y) = range(7)
@@ -37,16 +39,19 @@ class MoeDesc(ctypes.Structure):
         ("format", ctypes.c_int32), ("lora_rank", ctypes.c_int32), ("lora_scale", ctypes.c_float),
         ("act", ctypes.c_int32), ("tokens_per_tile", ctypes.c_int32),
         ("glu_alpha", ctypes.c_float), ("glu_limit", ctypes.c_float), ("glu_beta", ctypes.c_float),
+        ("gating", ctypes.c_int32),
     ]
 
 
-def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0, glu=None):
-    """glu None: SwiGLU; glu = (alpha, limit, beta): the clamped GLU (E4B_ACT_CLAMPED_GLU)."""
+def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0, glu=None, gating="topk"):
+    """glu None: SwiGLU; glu = (alpha, limit, beta): the clamped GLU (E4B_ACT_CLAMPED_GLU).
+    gating "topk" (softmax over the k picks) or "all" (full softmax, not renormalised)."""
     f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    g = GATINGS[gating] if isinstance(gating, str) else int(gating)
     if glu is None:
-        return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_SWIGLU, tokens_per_tile, 0.0, 0.0, 0.0)
+        return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_SWIGLU, tokens_per_tile, 0.0, 0.0, 0.0, g)
     a, lim, b = glu
-    return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_CLAMPED_GLU, tokens_per_tile, a, lim, b)
+    return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_CLAMPED_GLU, tokens_per_tile, a, lim, b, g)
 
 
 _LIB = None
@@ -59,8 +64,8 @@ _SIGS = {
     "e4b_quantize_nf4": ([_vp, _i64, _vp, _vp, _vp], _i32),
     "e4b_deinterleave_rows": ([_vp, _vp, _i32, _i32, _i64, _vp], _i32),
     "e4b_route_workspace_bytes": ([_i32, _i32, _i32], _sz),
-    "e4b_route": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
-    "e4b_route_noalloc": ([_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
+    "e4b_route": ([_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_route_noalloc": ([_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
     "e4b_moe_workspace_bytes": ([ctypes.POINTER(MoeDesc), _i32], _sz),
     "e4b_moe_workspace_region": ([ctypes.POINTER(MoeDesc), _i32, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz)], _i32),
     "e4b_moe_forward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -149,17 +154,17 @@ def e4b_route_workspace_bytes(T, E, k):
     return lib().e4b_route_workspace_bytes(T, E, k)
 
 
-def e4b_route(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_slot, ws, stream=None):
+def e4b_route(logits, T, E, k, gating, topk_ids, topk_w, expert_offsets, sorted_slot, ws, stream=None):
     _need_cuda(logits, topk_ids, topk_w, expert_offsets, sorted_slot, ws)
-    _check(lib().e4b_route(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
+    _check(lib().e4b_route(_ptr(logits), T, E, k, gating, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
                            _ptr(sorted_slot), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "e4b_route")
 
 
-def e4b_route_noalloc(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_slot, stream=None):
+def e4b_route_noalloc(logits, T, E, k, gating, topk_ids, topk_w, expert_offsets, sorted_slot, stream=None):
     """e4b_route with the library's fixed internal scratch instead of a caller workspace."""
     _need_cuda(logits, topk_ids, topk_w, expert_offsets, sorted_slot)
-    _check(lib().e4b_route_noalloc(_ptr(logits), T, E, k, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
+    _check(lib().e4b_route_noalloc(_ptr(logits), T, E, k, gating, _ptr(topk_ids), _ptr(topk_w), _ptr(expert_offsets),
                                    _ptr(sorted_slot), _stream(stream)), "e4b_route_noalloc")
 
 

@@ -37,16 +37,17 @@ def quantize_stack_nf4(w_f32: torch.Tensor, stream=None) -> PackedStack:
 
 class MoeLayer:
     def __init__(self, E, H, I, k, fmt, gate_up: PackedStack, down: PackedStack, lora_A=None, lora_B=None,
-                 lora_scale=0.0, tokens_per_tile=0, gu_bias=None, dn_bias=None, glu=None):
+                 lora_scale=0.0, tokens_per_tile=0, gu_bias=None, dn_bias=None, glu=None, gating="topk"):
         """gu_bias [E, 2I] / dn_bias [E, H] fp32 device tensors (or None) and glu = (alpha, limit, beta)
-        select the gpt-oss epilogue; gate_up rows must already be [gate | up] (see deinterleave_gate_up)."""
+        select the gpt-oss epilogue; gate_up rows must already be [gate | up] (see deinterleave_gate_up).
+        gating: "topk" (softmax over the k picks) or "all" (full softmax at the picks, not renormalised)."""
         self.E, self.H, self.I, self.k, self.fmt = E, H, I, k, fmt
         self.gate_up, self.down = gate_up, down
         self.lora_A, self.lora_B = lora_A, lora_B
         self.gu_bias, self.dn_bias = gu_bias, dn_bias
         self.lora_rank = 0 if lora_A is None else lora_A.shape[-1]
         self.lora_scale = lora_scale
-        self.desc = e4b.make_desc(E, H, I, k, fmt, self.lora_rank, lora_scale, tokens_per_tile, glu)
+        self.desc = e4b.make_desc(E, H, I, k, fmt, self.lora_rank, lora_scale, tokens_per_tile, glu, gating)
         self._ws = None
 
     def workspace(self, T, device):
@@ -172,7 +173,7 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
         bdn = torch.from_numpy(synth.normal_f32((E, H), w.bias_std, w.seed, "down_bias")).to(device)
     if w.interleaved:
         gu, bgu = deinterleave_gate_up(gu, bgu)
-    return MoeLayer(E, H, I, w.k, w.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu)
+    return MoeLayer(E, H, I, w.k, w.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu, w.gating)
 
 
 def synthetic_tokens(w: Workload, T, seed_offset=0):

@@ -81,6 +81,14 @@ enum { E4B_NF4 = 0, E4B_MXFP4 = 1 };   /* e4b_moe_desc.format */
  * The public gpt-oss release uses glu_alpha = 1.702, glu_limit = 7, glu_beta = 1. */
 enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 };
 
+/* Router gate weights (e4b_moe_desc.gating, e4b_route's gating argument).
+ * E4B_GATE_SOFTMAX_TOPK: softmax over the k selected logits (they sum to 1).
+ * E4B_GATE_SOFTMAX_ALL : softmax over all E logits, read at the k selected
+ *                        experts without renormalising (they sum to <= 1).
+ * The pages do not state the gating function; the first is the library's
+ * reading for the named families, the second the other common choice. */
+enum { E4B_GATE_SOFTMAX_TOPK = 0, E4B_GATE_SOFTMAX_ALL = 1 };
+
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st* e4b_stream;
 
@@ -103,6 +111,7 @@ typedef struct {
   float glu_alpha;         /* E4B_ACT_CLAMPED_GLU only: finite */
   float glu_limit;         /* E4B_ACT_CLAMPED_GLU only: > 0, +inf allowed (no clamp) */
   float glu_beta;          /* E4B_ACT_CLAMPED_GLU only: finite */
+  int32_t gating;          /* E4B_GATE_SOFTMAX_TOPK or E4B_GATE_SOFTMAX_ALL */
 } e4b_moe_desc;
 
 /* ABI version of the loaded library (E4B_ABI_VERSION it was built with). */
@@ -167,10 +176,11 @@ size_t e4b_route_workspace_bytes(int32_t T, int32_t E, int32_t k);
  * experts in one launch), [PKG] "Current measured position" (routing is
  * defined on given logits).
  *   logits         : [T, E] bf16, row-major       (device, read)
+ *   gating         : E4B_GATE_SOFTMAX_TOPK or E4B_GATE_SOFTMAX_ALL
  *   topk_ids       : [T, k] int32                 (device, written) ids by
  *                    (logit desc, id asc); -0 == +0
- *   topk_w         : [T, k] fp32                  (device, written) softmax of
- *                    the k selected logits
+ *   topk_w         : [T, k] fp32                  (device, written) gate
+ *                    weights as `gating` says
  *   expert_offsets : [E+1] int32                  (device, written) exclusive
  *                    prefix sum of per-expert slot counts
  *   sorted_slot    : [T*k] int32                  (device, written) slots
@@ -179,13 +189,13 @@ size_t e4b_route_workspace_bytes(int32_t T, int32_t E, int32_t k);
  * Integer outputs are deterministic and bit-exact.  T == 0 is a no-op that
  * still writes expert_offsets (all zero).
  */
-e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
+e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
                      int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
                      int32_t* sorted_slot, void* ws, size_t ws_bytes, e4b_stream stream);
 
 /*
- * e4b_route without a caller-provided workspace.  The paper has no
- * counterpart: this entry point exists for callers that cannot allocate
+ * e4b_route without a caller-provided workspace.  The described system has
+ * no counterpart: this entry point exists for callers that cannot allocate
  * device memory -- for instance a host runtime that owns all device memory
  * through its own pool and forbids cudaMalloc once running, or a serving loop
  * that must not risk an allocation that synchronises the device.
@@ -201,7 +211,7 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
  *   GPU (different streams, no ordering between them) race and corrupt each
  *   other's results: order them on one stream or with events.
  */
-e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k,
+e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
                              int32_t* topk_ids, float* topk_w, int32_t* expert_offsets,
                              int32_t* sorted_slot, e4b_stream stream);
 

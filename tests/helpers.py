@@ -124,6 +124,6 @@ def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=
     bgu, bdn = oracle_epilogue(w)
     ref, _ = omoe.moe_forward(x[rows], logits[rows], w.k, w.fmt, w.E, w.H, w.I, *ref_stacks,
                               lora_A_bits=A, lora_B_bits=B, lora_scale=w.lora_scale, gu_bias=bgu, dn_bias=bdn,
-                              glu=w.glu)
+                              glu=w.glu, gating=w.gating)
     got = bf16_to_f64(out)[rows]
     return assert_close_layer(got, ref, f"{w.name} T={T} tile={tokens_per_tile}"), lay, out

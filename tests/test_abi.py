@@ -45,9 +45,12 @@ def test_format_calls_reject_bad_sizes_and_pointers(L):
 
 
 def test_route_validation(L):
-    assert L.e4b_route(None, 4, 8, 9, None, None, None, None, None, 0, None) == e4b.E4B_ERR_INVALID_ARG
-    assert L.e4b_route(None, 4, 300, 2, None, None, None, None, None, 0, None) == e4b.E4B_ERR_UNSUPPORTED
-    assert L.e4b_route(None, 4, 8, 2, None, None, 256, None, 256, 1 << 20, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_route(None, 4, 8, 9, 0, None, None, None, None, None, 0, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_route(None, 4, 300, 2, 0, None, None, None, None, None, 0, None) == e4b.E4B_ERR_UNSUPPORTED
+    assert L.e4b_route(None, 4, 8, 2, 0, None, None, 256, None, 256, 1 << 20, None) == e4b.E4B_ERR_INVALID_ARG
+    # an unknown gating mode is refused before anything else is looked at
+    assert L.e4b_route(None, 4, 8, 2, 2, None, None, 256, None, 256, 1 << 20, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_route_noalloc(None, 4, 8, 2, -1, None, None, 256, None, None) == e4b.E4B_ERR_INVALID_ARG
     assert L.e4b_route_workspace_bytes(16, 8, 2) > 0
     assert L.e4b_route_workspace_bytes(16, 8, 9) == 0
 
@@ -67,7 +70,8 @@ def test_forward_validation_and_workspace(L):
                 # clamped GLU needs a positive limit and finite alpha / beta
                 e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(1.702, 0.0, 1.0)),
                 e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(float("nan"), 7.0, 1.0)),
-                e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(1.702, 7.0, float("inf")))]:
+                e4b.make_desc(8, 256, 128, 2, "mxfp4", glu=(1.702, 7.0, float("inf"))),
+                e4b.make_desc(8, 256, 128, 2, "mxfp4", gating=5)]:
         assert e4b.e4b_moe_workspace_bytes(bad, 64) == 0
     # the same shape is served by the tcgen05 tiles, and by the decode kernel at 2048
     assert e4b.e4b_moe_workspace_bytes(e4b.make_desc(8, 8192, 128, 2, "nf4"), 64) > 0

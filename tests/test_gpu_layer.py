@@ -155,6 +155,12 @@ def test_unclamped_glu_with_zero_bias_is_swiglu(tpt):
     assert torch.equal(glu.forward(xb, lb).float(), base.float())
 
 
+@pytest.mark.parametrize("tpt", [0, 8, 64])
+def test_full_softmax_gating_layer(tpt):
+    w = Workload("gate_all", "mxfp4", E=8, H=256, I=128, k=3, tokens=(90,), gating="all", seed=8)
+    run_and_compare(w, 90, tokens_per_tile=tpt)
+
+
 @pytest.mark.parametrize("row_bytes,offset", [(1440, 0), (90, 0), (4, 0), (16, 0), (64, 1)])
 def test_deinterleave_rows_bit_exact(row_bytes, offset):
     from oracle import moe as omoe

@@ -11,7 +11,7 @@ from oracle import route as oroute
 pytestmark = pytest.mark.gpu
 
 
-def _gpu_route(logits_bits, k):
+def _gpu_route(logits_bits, k, gating="topk"):
     dev = device()
     T, E = logits_bits.shape
     lg = torch.from_numpy(np.ascontiguousarray(logits_bits).view(np.int16)).to(dev)
@@ -20,15 +20,15 @@ def _gpu_route(logits_bits, k):
     off = torch.full((E + 1,), -7, dtype=torch.int32, device=dev)
     ss = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
     ws = torch.empty(e4b.e4b_route_workspace_bytes(T, E, k), dtype=torch.uint8, device=dev)
-    e4b.e4b_route(lg, T, E, k, ids, w, off, ss, ws)
+    e4b.e4b_route(lg, T, E, k, e4b.GATINGS[gating], ids, w, off, ss, ws)
     assert e4b.e4b_device_status(ws) == e4b.E4B_OK
     return (ids[:T * k].cpu().numpy().reshape(T, k), w[:T * k].cpu().numpy().reshape(T, k),
             off.cpu().numpy(), ss[:T * k].cpu().numpy())
 
 
-def _check(logits_bits, k):
-    ids, w, off, ss = _gpu_route(logits_bits, k)
-    r = oroute.route(logits_bits, k)
+def _check(logits_bits, k, gating="topk"):
+    ids, w, off, ss = _gpu_route(logits_bits, k, gating)
+    r = oroute.route(logits_bits, k, gating)
     assert np.array_equal(ids, r["ids"])
     assert np.array_equal(off, r["offsets"])
     assert np.array_equal(ss, r["sorted_slot"])
@@ -56,6 +56,18 @@ def test_route_all_tokens_one_expert():
     lg = np.zeros((3000, 16), np.float32)
     lg[:, 5] = 10.0
     _check(synth.to_bf16_bits(lg), 2)
+
+
+@pytest.mark.parametrize("T,E,k", [(64, 128, 8), (5, 5, 5), (1000, 32, 4), (2048, 128, 8), (300, 256, 8)])
+def test_route_full_softmax_gating(T, E, k):
+    # one routing block (T <= 128) and the multi-block path; k = E sums to 1
+    _check(synth.normal_bf16((T, E), 2.0, 0, f"groute{T}_{E}"), k, "all")
+
+
+def test_route_full_softmax_gating_ties():
+    g = np.random.default_rng(4)
+    vals = np.array([-1.0, -0.0, 0.0, 0.5, 2.0], np.float32)
+    _check(synth.to_bf16_bits(g.choice(vals, size=(500, 64))), 8, "all")
 
 
 def test_route_empty_batch():

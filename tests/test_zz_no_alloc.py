@@ -26,13 +26,13 @@ def _outputs(T, E, k, dev):
 def _with_workspace(lg, T, E, k, dev):
     ids, w, off, ss = _outputs(T, E, k, dev)
     ws = torch.empty(e4b.e4b_route_workspace_bytes(T, E, k), dtype=torch.uint8, device=dev)
-    e4b.e4b_route(lg, T, E, k, ids, w, off, ss, ws)
+    e4b.e4b_route(lg, T, E, k, 0, ids, w, off, ss, ws)
     return ids, w, off, ss
 
 
 def _without_workspace(lg, T, E, k, dev):
     ids, w, off, ss = _outputs(T, E, k, dev)
-    e4b.e4b_route_noalloc(lg, T, E, k, ids, w, off, ss)
+    e4b.e4b_route_noalloc(lg, T, E, k, 0, ids, w, off, ss)
     return ids, w, off, ss
 
 
