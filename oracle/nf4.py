@@ -32,6 +32,15 @@ contiguous dimension):
 
 Packing reading (pages silent): bitsandbytes' packed order, element 2j in the
 HIGH nibble of byte j, element 2j+1 in the low nibble.
+
+Double-quantised absmax ("experts4bit-qlora" package page, limits list: the
+absmax of an NF4 stack may be stored in bitsandbytes' nested form -- an
+offset, 8-bit codes and one fp32 per 256 values, about a quarter of the
+bytes -- and is expanded back to fp32 just in time for one layer).  The pages
+print neither the 8-bit code table nor the rounding of the expansion; this
+reading takes the 256-entry fp32 table as part of the stored form and
+expands, per absmax b, in fp32 with two roundings:
+absmax[b] = fl32(fl32(table[code[b]] * absmax2[b // 256]) + offset).
 """
 from statistics import NormalDist
 
@@ -112,3 +121,17 @@ def decode_nf4(packed, absmax, n):
     c = nf4_codebook().astype(np.float64)
     a = np.repeat(np.asarray(absmax, dtype=np.float32).astype(np.float64)[: n // BLOCK], BLOCK)
     return c[codes] * a
+
+
+DQ_BLOCK = 256
+
+
+def expand_absmax_dq(codes8, absmax2, offset, table):
+    """Nested-form absmax -> fp32 absmax [len(codes8)]: fl32(fl32(table[c] * absmax2[b // 256]) + offset)."""
+    c = np.asarray(codes8, dtype=np.uint8).reshape(-1)
+    t = np.asarray(table, dtype=np.float32).reshape(256)
+    s2 = np.asarray(absmax2, dtype=np.float32).reshape(-1)
+    blk = np.arange(c.size) // DQ_BLOCK
+    assert s2.size >= (c.size + DQ_BLOCK - 1) // DQ_BLOCK
+    prod = (t[c] * s2[blk]).astype(np.float32)           # fp32 product, one rounding
+    return (prod + np.float32(offset)).astype(np.float32)

@@ -204,3 +204,37 @@ def test_nf4_absmax_is_exact_max_and_scale_invariance():
     # scaling a block by a power of two changes absmax only
     packed2, absmax2 = nf4.quantize_nf4(x * np.float32(8.0))
     assert np.array_equal(packed, packed2) and np.array_equal(absmax2, absmax * 8)
+
+
+# ---------------------------------------------------------------- double-quantised absmax
+
+def test_expand_absmax_dq_exact_cases():
+    # a linear signed table j/127 (j = -127..128) keeps products of powers of two exact
+    table = (np.arange(256) - 127).astype(np.float32) / np.float32(127)
+    codes = np.array([127, 254, 0, 128, 200], np.uint8)
+    absmax2 = np.array([2.0 ** -3], np.float32)
+    out = nf4.expand_absmax_dq(codes, absmax2, np.float32(0.25), table)
+    expect = np.float32(0.25) + (codes.astype(np.int64) - 127).astype(np.float32) / np.float32(127) * np.float32(2 ** -3)
+    assert np.array_equal(out[:2], np.array([0.25, 0.25 + 2 ** -3], np.float32))     # codes 127 (0) and 254 (1)
+    assert out.dtype == np.float32 and np.allclose(out, expect, rtol=2e-7, atol=0)
+
+
+def test_expand_absmax_dq_second_level_blocks_are_256_long():
+    table = np.zeros(256, np.float32)
+    table[1] = 1.0
+    codes = np.ones(600, np.uint8)
+    absmax2 = np.array([1.0, 2.0, 4.0], np.float32)
+    out = nf4.expand_absmax_dq(codes, absmax2, 0.0, table)
+    assert np.array_equal(out[:256], np.ones(256, np.float32))
+    assert np.array_equal(out[256:512], np.full(256, 2.0, np.float32))
+    assert np.array_equal(out[512:], np.full(88, 4.0, np.float32))
+
+
+def test_expand_absmax_dq_rounds_product_then_sum():
+    # (1 + 2^-12)^2 = 1 + 2^-11 + 2^-24: the fp32 product ties to even at 1 + 2^-11, so adding -1 gives
+    # 2^-11; one fused rounding would keep 2^-11 + 2^-24
+    table = np.zeros(256, np.float32)
+    table[3] = np.float32(1.0 + 2.0 ** -12)
+    out = nf4.expand_absmax_dq(np.array([3], np.uint8), np.array([1.0 + 2.0 ** -12], np.float32), np.float32(-1.0),
+                               table)
+    assert out[0] == np.float32(2.0 ** -11)
