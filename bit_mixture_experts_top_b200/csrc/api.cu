@@ -40,8 +40,24 @@ __global__ void wait_timeout_probe_kernel(int32_t* status, uint64_t limit_ns) {
 
 struct ForwardLayout {
   size_t status, topk_ids, topk_w, offsets, chunk_off, block_counts, sorted_slot, slot_pos, x_sorted, xa, h, y;
+  size_t gu_absmax, dn_absmax;   // expanded double-quantised absmax (E4B_NF4_DQ only)
   size_t total;
 };
+
+// Absmax values of one stack [E, N, K] (one per 64 weights).
+size_t absmax_count(const e4b_moe_desc& d, bool gate_up) {
+  return static_cast<size_t>(d.E) * (gate_up ? 2 * static_cast<size_t>(d.I) : d.H) *
+         (gate_up ? d.H : d.I) / 64;
+}
+
+// The format the GEMM kernels see: a double-quantised stack runs as NF4 on its expanded absmax.
+int32_t gemm_format(int32_t format) { return format == E4B_NF4_DQ ? E4B_NF4 : format; }
+
+// A nested-form absmax description: every array present, the fp32 ones 4-byte aligned.
+bool valid_dq(const e4b_nf4_dq* q) {
+  return q && q->codes && q->absmax2 && q->offset && q->table && aligned(q->absmax2, 4) && aligned(q->offset, 4) &&
+         aligned(q->table, 4);
+}
 
 ForwardLayout forward_layout(const e4b_moe_desc& d, int32_t T) {
   const size_t R = static_cast<size_t>(T) * d.k;
@@ -65,6 +81,9 @@ ForwardLayout forward_layout(const e4b_moe_desc& d, int32_t T) {
   L.xa = take(d.lora_rank > 0 ? R * 128 : 0);
   L.h = take(R * d.I * 2);
   L.y = take(R * d.H * 4);
+  const bool dq = d.format == E4B_NF4_DQ;
+  L.gu_absmax = take(dq ? absmax_count(d, true) * 4 : 0);
+  L.dn_absmax = take(dq ? absmax_count(d, false) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -91,7 +110,7 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (!d || T < 0) return E4B_ERR_INVALID_ARG;
   if (d->E < 1 || d->E > kMaxExperts || d->k < 1 || d->k > d->E || d->k > kMaxTopK) return E4B_ERR_UNSUPPORTED;
   if (d->H < 64 || d->H % 64 != 0 || d->I < 64 || d->I % 64 != 0) return E4B_ERR_UNSUPPORTED;
-  if (d->format != E4B_NF4 && d->format != E4B_MXFP4) return E4B_ERR_UNSUPPORTED;
+  if (d->format != E4B_NF4 && d->format != E4B_MXFP4 && d->format != E4B_NF4_DQ) return E4B_ERR_UNSUPPORTED;
   if (d->act != E4B_ACT_SWIGLU && d->act != E4B_ACT_CLAMPED_GLU) return E4B_ERR_UNSUPPORTED;
   if (d->act == E4B_ACT_CLAMPED_GLU &&
       (!std::isfinite(d->glu_alpha) || !std::isfinite(d->glu_beta) || !(d->glu_limit > 0.0f)))
@@ -99,7 +118,8 @@ e4b_status validate_desc(const e4b_moe_desc* d, int32_t T) {
   if (d->lora_rank < 0 || d->lora_rank > kMaxLoraRank) return E4B_ERR_UNSUPPORTED;
   if (d->gating != E4B_GATE_SOFTMAX_TOPK && d->gating != E4B_GATE_SOFTMAX_ALL) return E4B_ERR_INVALID_ARG;
   const int tpt = d->tokens_per_tile;
-  if (tpt == 8 && !(skinny_gemm_supported(d->H, d->format) && skinny_gemm_supported(d->I, d->format)))
+  const int32_t gf = gemm_format(d->format);
+  if (tpt == 8 && !(skinny_gemm_supported(d->H, gf) && skinny_gemm_supported(d->I, gf)))
     return E4B_ERR_UNSUPPORTED;
   if (tpt != 0 && tpt != 8 && tpt != 32 && tpt != 64 && tpt != 128 && tpt != 192 && tpt != 256) return E4B_ERR_UNSUPPORTED;
   const int64_t R = static_cast<int64_t>(T) * d->k;
@@ -123,7 +143,8 @@ KernelChoice pick_kernel(const e4b_moe_desc& d, int32_t T) {
   const int64_t R = static_cast<int64_t>(T) * d.k;
   const int64_t active = R < d.E ? R : d.E;
   const int64_t avg = active > 0 ? (R + active - 1) / active : 1;
-  const bool decode_ok = skinny_gemm_supported(d.H, d.format) && skinny_gemm_supported(d.I, d.format);
+  const int32_t gf = gemm_format(d.format);
+  const bool decode_ok = skinny_gemm_supported(d.H, gf) && skinny_gemm_supported(d.I, gf);
   const int32_t chunk = avg <= 8 ? 8 : (avg <= 16 ? 16 : 32);
   if (d.tokens_per_tile == 8) return {true, chunk};
   if (d.tokens_per_tile) return {false, d.tokens_per_tile};
@@ -170,6 +191,16 @@ e4b_status e4b_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_
   if (n == 0) return E4B_OK;
   if (!codes || !scales || !out || !aligned(codes, 16) || !aligned(out, 16)) return E4B_ERR_INVALID_ARG;
   return launch_dequant_mxfp4(codes, scales, n, out, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? E4B_OK
+             : E4B_ERR_CUDA;
+}
+
+e4b_status e4b_expand_absmax_dq(const e4b_nf4_dq* dq, int64_t n, float* out, e4b_stream stream) {
+  if (n < 0) return E4B_ERR_INVALID_ARG;
+  if (n == 0) return E4B_OK;
+  if (!valid_dq(dq) || !out || !aligned(out, 4)) return E4B_ERR_INVALID_ARG;
+  return launch_expand_absmax_dq(dq->codes, dq->absmax2, dq->offset, dq->table, n, n, nullptr, out,
+                                 reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? E4B_OK
              : E4B_ERR_CUDA;
 }
@@ -249,6 +280,14 @@ e4b_status e4b_moe_workspace_region(const e4b_moe_desc* d, int32_t T, int32_t re
     case E4B_WS_X_SORTED: *offset = L.x_sorted; *bytes = R * d->H * 2; break;
     case E4B_WS_H: *offset = L.h; *bytes = R * d->I * 2; break;
     case E4B_WS_Y: *offset = L.y; *bytes = R * d->H * 4; break;
+    case E4B_WS_GU_ABSMAX:
+      *offset = L.gu_absmax;
+      *bytes = d->format == E4B_NF4_DQ ? absmax_count(*d, true) * 4 : 0;
+      break;
+    case E4B_WS_DN_ABSMAX:
+      *offset = L.dn_absmax;
+      *bytes = d->format == E4B_NF4_DQ ? absmax_count(*d, false) * 4 : 0;
+      break;
     default: return E4B_ERR_INVALID_ARG;
   }
   return E4B_OK;
@@ -267,10 +306,13 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   if (!ws || !aligned(ws, kAlign)) return E4B_ERR_INVALID_ARG;
   const ForwardLayout L = forward_layout(*d, T);
   if (ws_bytes < L.total) return E4B_ERR_INVALID_ARG;
+  const bool dq = d->format == E4B_NF4_DQ;
   if (T > 0) {
     if (!x || !logits || !gu_codes || !gu_scales || !dn_codes || !dn_scales || !out) return E4B_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gu_codes, 16) || !aligned(dn_codes, 16) ||
-        !aligned(gu_scales, 16) || !aligned(dn_scales, 16))
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gu_codes, 16) || !aligned(dn_codes, 16))
+      return E4B_ERR_INVALID_ARG;
+    if (dq ? !(valid_dq(static_cast<const e4b_nf4_dq*>(gu_scales)) && valid_dq(static_cast<const e4b_nf4_dq*>(dn_scales)))
+           : !(aligned(gu_scales, 16) && aligned(dn_scales, 16)))
       return E4B_ERR_INVALID_ARG;
     if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 2))) return E4B_ERR_INVALID_ARG;
     if ((gu_bias && !aligned(gu_bias, 4)) || (dn_bias && !aligned(dn_bias, 4))) return E4B_ERR_INVALID_ARG;
@@ -294,9 +336,11 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   uint16_t* xa = lora ? at<uint16_t>(ws, L.xa) : nullptr;
   uint16_t* h = at<uint16_t>(ws, L.h);
   float* y = at<float>(ws, L.y);
+  float* gu_absmax = at<float>(ws, L.gu_absmax);
+  float* dn_absmax = at<float>(ws, L.dn_absmax);
 
   GroupedGemmLaunch g;
-  g.fmt = d->format;
+  g.fmt = gemm_format(d->format);
   g.E = d->E;
   g.I = d->I;
   g.R = R;
@@ -321,13 +365,23 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         if (launch_gather(x, d->H, d->k, R, b.sorted_slot, b.topk_ids, d->E, x_sorted, lora_A, d->lora_rank,
                           d->lora_scale, xa, s) != cudaSuccess)
           return E4B_ERR_CUDA;
+        if (dq && T > 0) {   // the touched experts' absmax, expanded to fp32 for this forward
+          const e4b_nf4_dq* gq = static_cast<const e4b_nf4_dq*>(gu_scales);
+          const e4b_nf4_dq* dqs = static_cast<const e4b_nf4_dq*>(dn_scales);
+          const size_t ng = absmax_count(*d, true), nd = absmax_count(*d, false);
+          if (launch_expand_absmax_dq(gq->codes, gq->absmax2, gq->offset, gq->table, ng, ng / d->E,
+                                      b.expert_offsets, gu_absmax, s) != cudaSuccess ||
+              launch_expand_absmax_dq(dqs->codes, dqs->absmax2, dqs->offset, dqs->table, nd, nd / d->E,
+                                      b.expert_offsets, dn_absmax, s) != cudaSuccess)
+            return E4B_ERR_CUDA;
+        }
         break;
       case E4B_STAGE_GATE_UP: {
         g.mode = 0;
         g.N = 2 * d->I;
         g.K = d->H;
         g.codes = gu_codes;
-        g.scales = gu_scales;
+        g.scales = dq ? static_cast<const void*>(gu_absmax) : gu_scales;
         g.act = x_sorted;
         g.xa = xa;
         g.lora_B = lora_B;
@@ -343,7 +397,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.N = d->H;
         g.K = d->I;
         g.codes = dn_codes;
-        g.scales = dn_scales;
+        g.scales = dq ? static_cast<const void*>(dn_absmax) : dn_scales;
         g.act = h;
         g.xa = nullptr;
         g.lora_B = nullptr;

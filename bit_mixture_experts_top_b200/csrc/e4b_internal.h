@@ -57,6 +57,11 @@ cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, in
                                  cudaStream_t s);
 
 cudaError_t launch_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, cudaStream_t s);
+// absmax[b] = fl32(fl32(table[codes[b]] * absmax2[b / 256]) + *offset) for b < n; with expert_offsets,
+// blocks of experts (per_expert absmax each) that no row is routed to are left unwritten.
+cudaError_t launch_expand_absmax_dq(const uint8_t* codes, const float* absmax2, const float* offset,
+                                    const float* table, int64_t n, int64_t per_expert,
+                                    const int32_t* expert_offsets, float* out, cudaStream_t s);
 cudaError_t launch_deinterleave_rows(const void* in, void* out, int32_t E, int32_t I, int64_t row_bytes,
                                      cudaStream_t s);
 

@@ -174,6 +174,66 @@ cudaError_t launch_deinterleave_rows(const void* in, void* out, int32_t E, int32
   return cudaGetLastError();
 }
 
+// Double-quantised NF4 absmax ("experts4bit-qlora" limits list: bitsandbytes'
+// nested form -- offset, 8-bit codes, one fp32 per 256 values -- expanded to
+// fp32 just in time for one layer):
+//   absmax[b] = fl32(fl32(table[code[b]] * absmax2[b / 256]) + offset),
+// two explicit roundings (__fmul_rn / __fadd_rn, never contracted to an FMA).
+// With expert_offsets, blocks of experts that no routed row touches are
+// skipped: the GEMMs read only touched experts' absmax.  Four codes per thread
+// (one 32-bit load, one 16-byte store) when the sizes and pointers allow.
+__global__ void __launch_bounds__(256) expand_absmax_dq_kernel(const uint8_t* __restrict__ codes,
+                                                               const float* __restrict__ absmax2,
+                                                               const float* __restrict__ offset,
+                                                               const float* __restrict__ table, int64_t n,
+                                                               int64_t per_expert,
+                                                               const int32_t* __restrict__ expert_offsets,
+                                                               float* __restrict__ out, int vec4) {
+  __shared__ float s_table[256];
+  s_table[threadIdx.x] = __ldg(table + threadIdx.x);
+  const float off = __ldg(offset);
+  __syncthreads();
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (vec4) {
+    for (int64_t q = first; q < n / 4; q += step) {
+      const int64_t b = 4 * q;
+      if (expert_offsets) {
+        const int64_t e = b / per_expert;
+        if (__ldg(expert_offsets + e + 1) == __ldg(expert_offsets + e)) continue;
+      }
+      const uint32_t c4 = __ldg(reinterpret_cast<const uint32_t*>(codes) + q);
+      const float s2 = __ldg(absmax2 + b / 256);          // the four share a second-level block
+      float4 v;
+      v.x = __fadd_rn(__fmul_rn(s_table[c4 & 0xFFu], s2), off);
+      v.y = __fadd_rn(__fmul_rn(s_table[(c4 >> 8) & 0xFFu], s2), off);
+      v.z = __fadd_rn(__fmul_rn(s_table[(c4 >> 16) & 0xFFu], s2), off);
+      v.w = __fadd_rn(__fmul_rn(s_table[c4 >> 24], s2), off);
+      reinterpret_cast<float4*>(out)[q] = v;
+    }
+  } else {
+    for (int64_t b = first; b < n; b += step) {
+      if (expert_offsets) {
+        const int64_t e = b / per_expert;
+        if (__ldg(expert_offsets + e + 1) == __ldg(expert_offsets + e)) continue;
+      }
+      out[b] = __fadd_rn(__fmul_rn(s_table[__ldg(codes + b)], __ldg(absmax2 + b / 256)), off);
+    }
+  }
+}
+
+cudaError_t launch_expand_absmax_dq(const uint8_t* codes, const float* absmax2, const float* offset,
+                                    const float* table, int64_t n, int64_t per_expert,
+                                    const int32_t* expert_offsets, float* out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const bool vec4 = n % 4 == 0 && per_expert % 4 == 0 && reinterpret_cast<uintptr_t>(codes) % 4 == 0 &&
+                    reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  const int64_t items = vec4 ? n / 4 : n;
+  expand_absmax_dq_kernel<<<grid_for(items, 256, 8), 256, 0, s>>>(codes, absmax2, offset, table, n, per_expert,
+                                                                  expert_offsets, out, vec4 ? 1 : 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t n, uint16_t* out,
                                  cudaStream_t s) {
   const int64_t units = n / 8;

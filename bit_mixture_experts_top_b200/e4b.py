@@ -17,14 +17,15 @@ LIB_PATH = os.path.join(PKG, "libe4b.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "e4b.h")
 
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_UNSUPPORTED, E4B_ERR_CUDA, E4B_ERR_TIMEOUT = range(5)
-E4B_NF4, E4B_MXFP4 = 0, 1
+E4B_NF4, E4B_MXFP4, E4B_NF4_DQ = 0, 1, 2
 E4B_ACT_SWIGLU, E4B_ACT_CLAMPED_GLU = 0, 1
 E4B_GATE_SOFTMAX_TOPK, E4B_GATE_SOFTMAX_ALL = 0, 1
 GATINGS = {"topk": E4B_GATE_SOFTMAX_TOPK, "all": E4B_GATE_SOFTMAX_ALL}
 E4B_STAGE_ROUTE, E4B_STAGE_GATHER, E4B_STAGE_GATE_UP, E4B_STAGE_DOWN, E4B_STAGE_COMBINE = range(5)
 (E4B_WS_TOPK_IDS, E4B_WS_TOPK_W, E4B_WS_EXPERT_OFFSETS, E4B_WS_SORTED_SLOT, E4B_WS_X_SORTED, E4B_WS_H,
  E4B_WS_Y) = range(7)
-FORMATS = {"nf4": E4B_NF4, "mxfp4": E4B_MXFP4}
+FORMATS = {"nf4": E4B_NF4, "mxfp4": E4B_MXFP4, "nf4_dq": E4B_NF4_DQ}
+E4B_WS_GU_ABSMAX, E4B_WS_DN_ABSMAX = 7, 8
 
 
 class E4BError(RuntimeError):
@@ -54,6 +55,20 @@ def make_desc(E, H, I, k, fmt, lora_rank=0, lora_scale=0.0, tokens_per_tile=0, g
     return MoeDesc(E, H, I, k, f, lora_rank, lora_scale, E4B_ACT_CLAMPED_GLU, tokens_per_tile, a, lim, b, g)
 
 
+class Nf4DQ(ctypes.Structure):
+    """e4b_nf4_dq: a double-quantised absmax (device tensors codes u8, absmax2 f32, offset f32 [1], table f32
+    [256]); the tensors are kept alive with the struct."""
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax2", ctypes.c_void_p), ("offset", ctypes.c_void_p),
+                ("table", ctypes.c_void_p)]
+
+
+def make_nf4_dq(codes, absmax2, offset, table):
+    _need_cuda(codes, absmax2, offset, table)
+    q = Nf4DQ(codes.data_ptr(), absmax2.data_ptr(), offset.data_ptr(), table.data_ptr())
+    q.tensors = (codes, absmax2, offset, table)
+    return q
+
+
 _LIB = None
 _vp, _sz, _i32, _i64, _u32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32
 _SIGS = {
@@ -63,6 +78,7 @@ _SIGS = {
     "e4b_dequant_mxfp4": ([_vp, _vp, _i64, _vp, _vp], _i32),
     "e4b_quantize_nf4": ([_vp, _i64, _vp, _vp, _vp], _i32),
     "e4b_deinterleave_rows": ([_vp, _vp, _i32, _i32, _i64, _vp], _i32),
+    "e4b_expand_absmax_dq": ([ctypes.POINTER(Nf4DQ), _i64, _vp, _vp], _i32),
     "e4b_route_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "e4b_route": ([_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i32),
     "e4b_route_noalloc": ([_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp], _i32),
@@ -99,6 +115,8 @@ def header_functions():
 
 
 def _ptr(t):
+    if isinstance(t, Nf4DQ):         # host struct describing device arrays (E4B_NF4_DQ scales)
+        return ctypes.cast(ctypes.pointer(t), ctypes.c_void_p)
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
@@ -114,7 +132,7 @@ def _check(status, where):
 
 def _need_cuda(*ts):
     for t in ts:
-        if t is not None and not t.is_cuda:
+        if t is not None and not isinstance(t, Nf4DQ) and not t.is_cuda:
             raise ValueError("e4b: tensors must be CUDA tensors")
 
 
@@ -141,6 +159,12 @@ def e4b_quantize_nf4(x, n, codes, absmax, stream=None):
     _need_cuda(x, codes, absmax)
     _check(lib().e4b_quantize_nf4(_ptr(x), n, _ptr(codes), _ptr(absmax), _stream(stream)), "e4b_quantize_nf4")
     return codes, absmax
+
+
+def e4b_expand_absmax_dq(dq, n, out, stream=None):
+    _need_cuda(out)
+    _check(lib().e4b_expand_absmax_dq(ctypes.byref(dq), n, _ptr(out), _stream(stream)), "e4b_expand_absmax_dq")
+    return out
 
 
 def e4b_deinterleave_rows(inp, out, E, I, row_bytes, stream=None):

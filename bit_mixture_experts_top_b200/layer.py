@@ -18,7 +18,7 @@ from .workloads import Workload
 class PackedStack:
     """One fused expert stack [E, N, K] packed in 4 bits (device tensors)."""
     codes: torch.Tensor       # uint8 [E*N*K/2]
-    scales: torch.Tensor      # NF4: fp32 [E*N*K/64]; MXFP4: uint8 [E*N*K/32]
+    scales: object            # NF4: fp32 [E*N*K/64]; MXFP4: uint8 [E*N*K/32]; "nf4_dq": an e4b.Nf4DQ
     E: int
     N: int
     K: int
@@ -163,6 +163,11 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
                                                                         "gate_up")).to(device))
         dn = quantize_stack_nf4(torch.from_numpy(synth.stack_normal_f32(E, H, I, w.weight_std, w.seed,
                                                                         "down")).to(device))
+        if w.absmax_dq:   # the codes stay; the absmax is replaced by a synthetic nested-form one
+            gu = PackedStack(gu.codes, nf4_dq_tensors(E, 2 * I * H // 64, w.seed, "gate_up_absmax", device),
+                             E, 2 * I, H, "nf4_dq")
+            dn = PackedStack(dn.codes, nf4_dq_tensors(E, H * I // 64, w.seed, "down_absmax", device),
+                             E, H, I, "nf4_dq")
     A = B = None
     if w.lora_rank:
         A = bits_tensor(synth.normal_bf16((E, H, w.lora_rank), 1.0 / w.lora_rank, w.seed, "lora_A"), device)
@@ -173,7 +178,14 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
         bdn = torch.from_numpy(synth.normal_f32((E, H), w.bias_std, w.seed, "down_bias")).to(device)
     if w.interleaved:
         gu, bgu = deinterleave_gate_up(gu, bgu)
-    return MoeLayer(E, H, I, w.k, w.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu, w.gating)
+    return MoeLayer(E, H, I, w.k, gu.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu, w.gating)
+
+
+def nf4_dq_tensors(E, n_per_expert, seed, name, device):
+    """The seeded nested-form absmax of a stack as an e4b.Nf4DQ over device tensors."""
+    codes, absmax2, offset, table = synth.nf4_dq_absmax(E, n_per_expert, seed, name)
+    t = [torch.from_numpy(a).to(device) for a in (codes, absmax2, offset, table)]
+    return e4b.make_nf4_dq(*t)
 
 
 def synthetic_tokens(w: Workload, T, seed_offset=0):

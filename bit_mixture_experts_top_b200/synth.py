@@ -15,6 +15,8 @@ Recipe (all streams keyed by ``seed`` and a tensor name):
 * LoRA: A ~ N(0, 1/r), B ~ N(0, 0.01) in bf16 (the second parameter is read
   as a standard deviation);
 * gpt-oss epilogue biases: fp32 N(0, std), std chosen per test;
+* double-quantised NF4 absmax: uniform 8-bit codes, U[0.01, 0.03] second-level
+  scales, offset 0.05, a linear code table over [-1, 1];
 * skewed routing: logits log p_e + Gumbel(0, 1) with p_e proportional to
   rank**-s over a seeded permutation of the experts, so a top-k pick is a
   Gumbel-top-k draw without replacement and expert load is Zipf(s) skewed.
@@ -46,6 +48,18 @@ def normal_bf16(shape, std, seed, name):
 def normal_f32(shape, std, seed, name):
     """fp32 N(0, std) values (biases of the gpt-oss epilogue)."""
     return rng(seed, name).standard_normal(shape, dtype=np.float32) * np.float32(std)
+
+
+def nf4_dq_absmax(E, n_per_expert, seed, name):
+    """Nested-form (double-quantised) absmax of a stack: 8-bit codes uniform over 0..255 (drawn per expert),
+    fp32 second-level scales U[0.01, 0.03] per 256 values, offset 0.05 and the fp32 code table
+    linspace(-1, 1, 256); the absmax it describes lies in [0.02, 0.08], the magnitude of N(0, 0.02) weights'."""
+    codes = np.empty((E, n_per_expert), dtype=np.uint8)
+    for e in range(E):
+        codes[e] = rng(seed, name + "_codes", e).integers(0, 256, size=n_per_expert, dtype=np.uint8)
+    n = E * n_per_expert
+    absmax2 = rng(seed, name + "_absmax2").uniform(0.01, 0.03, size=(n + 255) // 256).astype(np.float32)
+    return codes.reshape(-1), absmax2, np.array([0.05], np.float32), np.linspace(-1.0, 1.0, 256, dtype=np.float32)
 
 
 def expert_normal_f32(e, N, K, std, seed, name):

@@ -27,6 +27,7 @@ class Workload:
     bias_std: float = 0.0                 # > 0: per-expert fp32 biases N(0, bias_std) on both stacks
     interleaved: bool = False             # gate_up drawn with gate/up rows interleaved, de-interleaved at load
     gating: str = "topk"                  # router weights: "topk" (softmax over the picks) or "all"
+    absmax_dq: bool = False               # NF4: absmax stored double-quantised (nested form)
     seed: int = 0
     notes: str = field(default="", compare=False)
 

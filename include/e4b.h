@@ -72,7 +72,25 @@ typedef enum {
   E4B_ERR_TIMEOUT = 4        /* a bounded device-side wait ran out (reported by e4b_device_status) */
 } e4b_status;
 
-enum { E4B_NF4 = 0, E4B_MXFP4 = 1 };   /* e4b_moe_desc.format */
+/* e4b_moe_desc.format.  E4B_NF4_DQ is NF4 whose absmax is stored double-quantised
+ * (e4b_nf4_dq below); the forward expands it to fp32 and runs as E4B_NF4. */
+enum { E4B_NF4 = 0, E4B_MXFP4 = 1, E4B_NF4_DQ = 2 };
+
+/*
+ * Double-quantised NF4 absmax: [PKG] limits list -- bitsandbytes' nested form
+ * of an NF4 stack's fp32 absmax (an offset, 8-bit codes and one fp32 per 256
+ * values, about a quarter of the bytes), expanded back to fp32 just in time.
+ * The pages give neither the 8-bit code table nor the expansion's rounding;
+ * the table is part of the stored form here and the expansion is, for
+ * absmax b,  fl32(fl32(table[codes[b]] * absmax2[b / 256]) + *offset)
+ * (two roundings, no fused multiply-add).  All four are device pointers.
+ */
+typedef struct {
+  const uint8_t* codes;    /* [n_absmax] 8-bit codes */
+  const float* absmax2;    /* [ceil(n_absmax / 256)] fp32 second-level scales, 4-byte aligned */
+  const float* offset;     /* [1] fp32, 4-byte aligned */
+  const float* table;      /* [256] fp32 code table, 4-byte aligned */
+} e4b_nf4_dq;
 /* e4b_moe_desc.act.  E4B_ACT_SWIGLU: h = silu(gate) * up, silu(z) = z / (1 + e^-z).
  * E4B_ACT_CLAMPED_GLU (gpt-oss, [MX] "Why it happens"; the pages give no formula or
  * constants, so this is the library's reading, with the constants as parameters):
@@ -153,6 +171,15 @@ e4b_status e4b_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* ab
                             e4b_stream stream);
 
 /*
+ * Double-quantised absmax -> fp32 (the read path's expansion on its own).
+ *   dq  : host struct describing the device arrays (see e4b_nf4_dq)
+ *   n   : absmax values, >= 0
+ *   out : n fp32 (device, written), 4-byte aligned
+ * Bit-exact: out[b] = fl32(fl32(table[codes[b]] * absmax2[b / 256]) + *offset).
+ */
+e4b_status e4b_expand_absmax_dq(const e4b_nf4_dq* dq, int64_t n, float* out, e4b_stream stream);
+
+/*
  * gpt-oss gate_up de-interleave (load-time layout step).  [MX] "Why it
  * happens" (interleaved gate/up rows), "Which project solves it" (the gpt-oss
  * module de-interleaves them).
@@ -228,6 +255,8 @@ size_t e4b_moe_workspace_bytes(const e4b_moe_desc* d, int32_t T);
  *   logits    : [T, E] bf16                            (device, read)
  *   gu_codes  : [E, 2I, H] packed 4-bit (E*2I*H/2 bytes, 16-byte aligned)
  *   gu_scales : NF4 fp32 absmax [E*2I*H/64] or MXFP4 E8M0 bytes [E*2I*H/32]
+ *               (device, 16-byte aligned); for E4B_NF4_DQ a HOST pointer to
+ *               an e4b_nf4_dq describing the stack's E*2I*H/64 absmax
  *   dn_codes  : [E, H, I] packed 4-bit;  dn_scales as gu_scales for [E, H, I]
  *   lora_A    : [E, H, r] bf16 or NULL;  lora_B : [E, r, 2I] bf16 or NULL
  *               (both or neither, and r == d->lora_rank)
@@ -253,7 +282,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, int32_t T, const uint16_t* x,
 /* Stages of e4b_moe_forward, in order. */
 enum {
   E4B_STAGE_ROUTE = 0,     /* clears the status word; top-k, histogram, stable permute */
-  E4B_STAGE_GATHER = 1,    /* routed rows in expert order (+ LoRA left factor x.A_e) */
+  E4B_STAGE_GATHER = 1,    /* routed rows in expert order (+ LoRA left factor x.A_e; E4B_NF4_DQ: the
+                              touched experts' absmax expanded to fp32) */
   E4B_STAGE_GATE_UP = 2,   /* grouped gate_up GEMM with dequant, LoRA delta, bias, activation -> h */
   E4B_STAGE_DOWN = 3,      /* grouped down GEMM with dequant (+ bias) -> y */
   E4B_STAGE_COMBINE = 4    /* out[t] = sum_j w[t,j] * y[t,j] */
@@ -280,7 +310,9 @@ enum {
   E4B_WS_SORTED_SLOT = 3,  /* int32 [T*k] */
   E4B_WS_X_SORTED = 4,     /* bf16  [T*k, H] */
   E4B_WS_H = 5,            /* bf16  [T*k, I]  act(gate, up) per routed row */
-  E4B_WS_Y = 6             /* fp32  [T*k, H]  down output per routed row */
+  E4B_WS_Y = 6,            /* fp32  [T*k, H]  down output per routed row */
+  E4B_WS_GU_ABSMAX = 7,    /* fp32  [E*2I*H/64] expanded gate_up absmax (E4B_NF4_DQ; touched experts only) */
+  E4B_WS_DN_ABSMAX = 8     /* fp32  [E*H*I/64]  expanded down absmax (E4B_NF4_DQ; touched experts only) */
 };
 
 /* Byte offset and size of one intermediate of e4b_moe_forward's workspace. */

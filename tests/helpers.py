@@ -65,17 +65,24 @@ def oracle_stacks(w, experts):
         for e in experts:
             gc[e], gs[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, 2 * I, H, w.weight_std, w.seed, "gate_up"))
             dc[e], ds[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, H, I, w.weight_std, w.seed, "down"))
+        if w.absmax_dq:   # the stored absmax is the nested form's expansion
+            gs = onf4.expand_absmax_dq(*synth.nf4_dq_absmax(E, 2 * I * H // 64, w.seed, "gate_up_absmax"))
+            ds = onf4.expand_absmax_dq(*synth.nf4_dq_absmax(E, H * I // 64, w.seed, "down_absmax"))
     return gc.reshape(-1), gs.reshape(-1), dc.reshape(-1), ds.reshape(-1)
 
 
-def check_nf4_stacks_equal(lay, w, experts, ref):
+def check_nf4_stacks_equal(lay, w, experts, ref, T):
     """The device-quantised stacks must equal the oracle's bit for bit on these experts."""
     gc, gs, dc, ds = ref
     E, H, I = w.E, w.H, w.I
     g_codes = lay.gate_up.codes.view(E, -1)
-    g_abs = lay.gate_up.scales.view(E, -1)
     d_codes = lay.down.codes.view(E, -1)
-    d_abs = lay.down.scales.view(E, -1)
+    if w.absmax_dq:   # the forward's expansion of the touched experts' absmax, in its workspace
+        g_abs = lay.region(T, e4b.E4B_WS_GU_ABSMAX, torch.float32).view(E, -1)
+        d_abs = lay.region(T, e4b.E4B_WS_DN_ABSMAX, torch.float32).view(E, -1)
+    else:
+        g_abs = lay.gate_up.scales.view(E, -1)
+        d_abs = lay.down.scales.view(E, -1)
     for e in experts:
         assert np.array_equal(g_codes[e].cpu().numpy(), gc.reshape(E, -1)[e])
         assert np.array_equal(g_abs[e].cpu().numpy().view(np.uint32), gs.reshape(E, -1)[e].view(np.uint32))
@@ -119,7 +126,7 @@ def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=
         gc, gs, dc, ds = ref_stacks
         ref_stacks = (omoe.deinterleave_rows(gc, w.E, w.I), omoe.deinterleave_rows(gs, w.E, w.I), dc, ds)
     if w.fmt == "nf4":
-        check_nf4_stacks_equal(lay, w, experts, ref_stacks)
+        check_nf4_stacks_equal(lay, w, experts, ref_stacks, T)
     A, B = oracle_lora(w)
     bgu, bdn = oracle_epilogue(w)
     ref, _ = omoe.moe_forward(x[rows], logits[rows], w.k, w.fmt, w.E, w.H, w.I, *ref_stacks,

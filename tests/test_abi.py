@@ -90,6 +90,23 @@ def test_forward_validation_and_workspace(L):
     assert L.e4b_debug_wait_timeout(2_000_000_000, 256, 4096, None) == e4b.E4B_ERR_INVALID_ARG
 
 
+def test_expand_absmax_dq_validation(L):
+    q = e4b.Nf4DQ(256, 256, 256, 256)
+    assert L.e4b_expand_absmax_dq(ctypes.byref(q), 0, None, None) == e4b.E4B_OK          # nothing to do
+    assert L.e4b_expand_absmax_dq(ctypes.byref(q), -1, 256, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_expand_absmax_dq(None, 16, 256, None) == e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_expand_absmax_dq(ctypes.byref(e4b.Nf4DQ(256, None, 256, 256)), 16, 256, None) == \
+        e4b.E4B_ERR_INVALID_ARG
+    assert L.e4b_expand_absmax_dq(ctypes.byref(e4b.Nf4DQ(256, 257, 256, 256)), 16, 256, None) == \
+        e4b.E4B_ERR_INVALID_ARG                                                           # misaligned fp32
+    # a double-quantised layer's workspace holds the two expanded absmax arrays
+    d, dq = e4b.make_desc(8, 256, 128, 2, "nf4"), e4b.make_desc(8, 256, 128, 2, "nf4_dq")
+    extra = e4b.e4b_moe_workspace_bytes(dq, 64) - e4b.e4b_moe_workspace_bytes(d, 64)
+    assert extra == 8 * 2 * 128 * 256 // 64 * 4 + 8 * 256 * 128 // 64 * 4
+    assert e4b.e4b_moe_workspace_region(dq, 64, e4b.E4B_WS_GU_ABSMAX)[1] == 8 * 2 * 128 * 256 // 64 * 4
+    assert e4b.e4b_moe_workspace_region(d, 64, e4b.E4B_WS_DN_ABSMAX)[1] == 0
+
+
 def test_deinterleave_validation(L):
     # sizes and overlap are checked on the host; empty inputs are a no-op (nothing launched)
     assert L.e4b_deinterleave_rows(None, None, 0, 64, 1440, None) == e4b.E4B_OK

@@ -161,6 +161,36 @@ def test_full_softmax_gating_layer(tpt):
     run_and_compare(w, 90, tokens_per_tile=tpt)
 
 
+# ---------------------------------------------------------------- double-quantised NF4 absmax
+
+@pytest.mark.parametrize("n", [1000, 4096, 7])
+def test_expand_absmax_dq_bit_exact(n):
+    from oracle import nf4 as onf4
+    dev = device()
+    g = np.random.default_rng(n)
+    codes = g.integers(0, 256, size=n, dtype=np.uint8)
+    absmax2 = g.uniform(0.001, 0.1, size=(n + 255) // 256).astype(np.float32)
+    offset = np.array([g.uniform(0.01, 0.1)], np.float32)
+    table = np.sort(g.standard_normal(256).astype(np.float32))
+    dq = e4b.make_nf4_dq(*[torch.from_numpy(a).to(dev) for a in (codes, absmax2, offset, table)])
+    out = torch.full((n,), float("nan"), dtype=torch.float32, device=dev)
+    e4b.e4b_expand_absmax_dq(dq, n, out)
+    ref = onf4.expand_absmax_dq(codes, absmax2, offset[0], table)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("tpt", [0, 8, 64])
+def test_nf4_double_quantised_absmax_layer(tpt):
+    # the forward expands the touched experts' absmax (checked bit for bit) and runs as NF4 on it
+    w = Workload("nf4_dq", "nf4", E=8, H=320, I=192, k=2, tokens=(60,), absmax_dq=True, seed=9)
+    run_and_compare(w, 60, tokens_per_tile=tpt)
+
+
+def test_qwen3_nf4_double_quantised_absmax_decode_sampled():
+    w = Workload("qwen3_dq", "nf4", E=128, H=2048, I=768, k=8, tokens=(64,), absmax_dq=True)
+    run_and_compare(w, 64, sample=np.arange(0, 64, 8))
+
+
 @pytest.mark.parametrize("row_bytes,offset", [(1440, 0), (90, 0), (4, 0), (16, 0), (64, 1)])
 def test_deinterleave_rows_bit_exact(row_bytes, offset):
     from oracle import moe as omoe
