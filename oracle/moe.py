@@ -53,7 +53,7 @@ import numpy as np
 from .bf16 import bf16_bits_to_f64
 from .mxfp4 import decode_mxfp4
 from .nf4 import decode_nf4
-from .route import route
+from .route import route_values
 
 NF4 = "nf4"
 MXFP4 = "mxfp4"
@@ -107,18 +107,35 @@ def moe_forward(x_bits, logits_bits, k, fmt, E, H, I, gu_codes, gu_scales, dn_co
     stock SwiGLU silu(gate) * up.  gating selects the router weights (:func:`oracle.route.route`).
     """
     x = bf16_bits_to_f64(np.asarray(x_bits, dtype=np.uint16)).reshape(-1, H)
+    logits = bf16_bits_to_f64(np.asarray(logits_bits, dtype=np.uint16)).reshape(x.shape[0], E)
+    A = B = None
+    if lora_A_bits is not None:
+        A = bf16_bits_to_f64(np.asarray(lora_A_bits, dtype=np.uint16))
+        B = bf16_bits_to_f64(np.asarray(lora_B_bits, dtype=np.uint16))
+    return moe_forward_values(x, logits, k, fmt, E, H, I, gu_codes, gu_scales, dn_codes, dn_scales, A, B,
+                              lora_scale, gu_bias, dn_bias, glu, gating)
+
+
+def lora_factors(A, B, E, H, I):
+    """LoRA factors as fp64 A [E, H, r] and B [E, r, 2I] (None when there is no adapter)."""
+    if A is None:
+        return None, None
+    A = np.asarray(A, dtype=np.float64)
+    rank = A.size // (E * H)
+    return A.reshape(E, H, rank), np.asarray(B, dtype=np.float64).reshape(E, rank, 2 * I)
+
+
+def moe_forward_values(x, logits, k, fmt, E, H, I, gu_codes, gu_scales, dn_codes, dn_scales, A=None, B=None,
+                       lora_scale=0.0, gu_bias=None, dn_bias=None, glu=None, gating="topk"):
+    """:func:`moe_forward` on fp64 values: x [T, H], logits [T, E], LoRA A [E, H, r] / B [E, r, 2I] or None."""
+    x = np.asarray(x, dtype=np.float64).reshape(-1, H)
     T = x.shape[0]
-    r = route(np.asarray(logits_bits, dtype=np.uint16).reshape(T, E), k, gating)
+    r = route_values(np.asarray(logits, dtype=np.float64).reshape(T, E), k, gating)
     offsets, sorted_slot = r["offsets"], r["sorted_slot"]
     x_sorted = x[sorted_slot // k]                       # step 2: permute
     y_sorted = np.zeros((T * k, H), dtype=np.float64)
-    lora = lora_A_bits is not None
-    if lora:
-        A = bf16_bits_to_f64(np.asarray(lora_A_bits, dtype=np.uint16))
-        B = bf16_bits_to_f64(np.asarray(lora_B_bits, dtype=np.uint16))
-        rank = A.size // (E * H)
-        A = A.reshape(E, H, rank)
-        B = B.reshape(E, rank, 2 * I)
+    A, B = lora_factors(A, B, E, H, I)
+    lora = A is not None
     for e in range(E):                                   # step 3: per expert
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if lo == hi:

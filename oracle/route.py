@@ -73,7 +73,12 @@ def route(logits_bits, k, gating="topk"):
 
     gating "topk": softmax over the k selected logits; "all": softmax over all E, top k kept as they are.
     """
-    logits = bf16_bits_to_f64(np.asarray(logits_bits, dtype=np.uint16))
+    return route_values(bf16_bits_to_f64(np.asarray(logits_bits, dtype=np.uint16)), k, gating)
+
+
+def route_values(logits, k, gating="topk"):
+    """:func:`route` on fp64 logit values [T, E]."""
+    logits = np.asarray(logits, dtype=np.float64)
     T, E = logits.shape
     assert 1 <= k <= E and gating in ("topk", "all")
     ids = topk_select(logits, k) if T else np.zeros((0, k), np.int32)
