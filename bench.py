@@ -303,11 +303,12 @@ def bench_e4b(args, world, rank, local):
     barrier()
     torch.cuda.synchronize()
     sampler.start()
-    t_start.record()
-    for _ in range(K):
-        g_fwd.replay()
-    t_end.record()
-    torch.cuda.synchronize()
+    with torch.cuda.nvtx.range(f"timed: {K} forwards"):      # NVTX ranges mark the bench's phases for nsys
+        t_start.record()
+        for _ in range(K):
+            g_fwd.replay()
+        t_end.record()
+        torch.cuda.synchronize()
     clocks = sampler.summary()
     barrier()
     total_ms = t_start.elapsed_time(t_end)
@@ -327,9 +328,10 @@ def bench_e4b(args, world, rank, local):
 
     # the dominant kernel, launch by launch (touched weights per launch exceed L2: no flush needed)
     n_stage = min(K, 500)
-    gu_ms = max_over_ranks(time_graph(g_gu, n_stage))
-    dn_ms = max_over_ranks(time_graph(g_dn, n_stage))
-    small_ms = {nm: max_over_ranks(time_graph(g, n_stage)) for nm, g in g_small.items()}
+    with torch.cuda.nvtx.range("per-stage timing"):
+        gu_ms = max_over_ranks(time_graph(g_gu, n_stage))
+        dn_ms = max_over_ranks(time_graph(g_dn, n_stage))
+        small_ms = {nm: max_over_ranks(time_graph(g, n_stage)) for nm, g in g_small.items()}
     if e4b.e4b_device_status(ws) != e4b.E4B_OK:
         raise RuntimeError("device status reported an error in the timed region")
     del g_fwd, g_gu, g_dn, g_small
@@ -344,11 +346,12 @@ def bench_e4b(args, world, rank, local):
         hf.run()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        hf.run()
-    e1.record()
-    torch.cuda.synchronize()
+    with torch.cuda.nvtx.range(f"end to end: {e2e_steps} host-to-host forwards"):
+        e0.record()
+        for _ in range(e2e_steps):
+            hf.run()
+        e1.record()
+        torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
     barrier()
     h2d_bytes = int(hf.x.numel() * 2 + hf.logits.numel() * 2)
