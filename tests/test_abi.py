@@ -1,6 +1,8 @@
 """CPU checks of the C ABI: the library loads, exports every declared entry
-point, its NF4 table equals the oracle's bit for bit, and host-side argument
-validation rejects bad calls before anything touches a GPU."""
+point, the Python binding's argument lists and struct layouts match the header
+(the layouts read from a host program gcc builds against it), its NF4 table
+equals the oracle's bit for bit, and host-side argument validation rejects bad
+calls before anything touches a GPU."""
 import ctypes
 
 import numpy as np
@@ -115,3 +117,44 @@ def test_deinterleave_validation(L):
     assert L.e4b_deinterleave_rows(None, 512, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG
     assert L.e4b_deinterleave_rows(256, 256 + 16, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG   # overlap
     assert L.e4b_deinterleave_rows(256 + 16, 256, 1, 1, 16, None) == e4b.E4B_ERR_INVALID_ARG
+
+
+def _header_params():
+    """{function: number of parameters} from the prototypes in include/e4b.h."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", open(e4b.HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(e4b_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    counts = _header_params()
+    assert set(counts) == set(e4b._SIGS)
+    for name, (args, _) in e4b._SIGS.items():
+        assert len(args) == counts[name], name
+
+
+def test_binding_structs_match_the_c_layout(tmp_path):
+    # compile a host program against the header and compare sizes and field offsets with ctypes
+    import subprocess
+    fields = {"e4b_moe_desc": e4b.MoeDesc, "e4b_nf4_dq": e4b.Nf4DQ}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "e4b.h"', "int main(void) {"]
+    for cname, py in fields.items():
+        lines.append(f'  printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in py._fields_:
+            lines.append(f'  printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    inc = str(__import__("pathlib").Path(e4b.HEADER).parent)
+    subprocess.run(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], check=True, capture_output=True,
+                                                 text=True).stdout.splitlines())
+    for cname, py in fields.items():
+        assert int(got[cname]) == ctypes.sizeof(py), cname
+        for f, _ in py._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
