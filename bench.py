@@ -76,7 +76,7 @@ class ClockSampler(threading.Thread):
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
                0x2: "applications_clocks_setting"}
 
-    def __init__(self, gpu_index, period_s=0.002):
+    def __init__(self, gpu_index, period_s=0.0002):
         super().__init__(daemon=True)
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.stop_evt, self.err = period_s, threading.Event(), None
@@ -115,6 +115,138 @@ class ClockSampler(threading.Thread):
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
                 **({"note": self.err} if self.err else {})}
+
+
+# every layer configuration the metric is quoted on (the tiny layer is a correctness case only)
+CONFIGS = [("qwen3_30b_a3b_nf4_decode", 1), ("qwen3_30b_a3b_nf4_decode", 8), ("qwen3_30b_a3b_nf4_decode", 32),
+           ("qwen3_30b_a3b_nf4_decode", 64), ("qwen3_30b_a3b_nf4_lora", 512), ("gptoss_20b_mxfp4", 1),
+           ("gptoss_20b_mxfp4", 16), ("gptoss_20b_mxfp4", 4096), ("gptoss_120b_mxfp4_zipf", 16384)]
+ROTATE_BYTES = 4 * L2_BYTES      # decode layers rotate over weight copies until this much is touched per pass
+MAX_COPIES = 24
+
+
+def bench_configs(dev, peaks, max_over_ranks, target_s=0.4):
+    """Every configuration of CONFIGS, timed as CUDA-graph replays of the whole forward.
+
+    Decode-sized layers touch less than L2 holds, so one pass replays the layer over several copies of its
+    packed stacks (identical bytes at distinct addresses, like consecutive layers of a model) until a pass
+    touches ROTATE_BYTES; the time per layer is the pass time over the copies.  The gate_up and down
+    launches are timed the same way on their own.  Decode-class layers report weight-stream GB/s against
+    the HBM peak, prefill-class ones TFLOP/s (real routed rows only) against the bf16 burst peak."""
+    import torch
+    from bit_mixture_experts_top_b200 import e4b, layer
+    from bit_mixture_experts_top_b200.workloads import WORKLOADS
+
+    rows, built = [], {}
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    for wname, T in CONFIGS:
+        w = WORKLOADS[wname]
+        key = (w.fmt, w.E, w.H, w.I, w.k, w.exp_range, w.weight_std, w.seed)
+        if key not in built:
+            built.clear()
+            torch.cuda.empty_cache()
+            built[key] = layer.synthetic_layer(w, dev)
+        base = built[key]
+        A, B = layer.synthetic_lora(w, dev)
+        lay = layer.MoeLayer(w.E, w.H, w.I, w.k, w.fmt, base.gate_up, base.down, A, B, w.lora_scale)
+        x_np, lg_np = layer.synthetic_tokens(w, T)
+        x, lg = layer.bits_tensor(x_np, dev), layer.bits_tensor(lg_np, dev)
+        out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+        ws = lay.workspace(T, dev)
+        lay.forward(x, lg, out)
+        torch.cuda.synchronize()
+        offs = lay.region(T, e4b.E4B_WS_EXPERT_OFFSETS, torch.int32).cpu().numpy()
+        touched = int(np.count_nonzero(np.diff(offs)))
+        R = T * w.k
+        wbytes = touched * (w.gate_up_bytes_per_expert() + w.down_bytes_per_expert())
+        lora_bytes = touched * (w.H + 2 * w.I) * w.lora_rank * 2
+        gu_bytes = touched * w.gate_up_bytes_per_expert() + R * w.H * 2 + R * w.I * 2 + lora_bytes
+        dn_bytes = touched * w.down_bytes_per_expert() + R * w.I * 2 + R * w.H * 4
+        gu_flops = 2 * R * w.H * 2 * w.I + (2 * R * (w.H + 2 * w.I) * w.lora_rank if w.lora_rank else 0)
+        dn_flops = 2 * R * w.I * w.H
+        tensor = gu_flops / gu_bytes > ridge
+        copies = 1 if wbytes >= ROTATE_BYTES else min(MAX_COPIES, -(-ROTATE_BYTES // max(wbytes, 1)))
+        layers = [lay]
+        for _ in range(copies - 1):
+            gu = layer.PackedStack(lay.gate_up.codes.clone(), lay.gate_up.scales.clone(), w.E, 2 * w.I, w.H, w.fmt)
+            dn = layer.PackedStack(lay.down.codes.clone(), lay.down.scales.clone(), w.E, w.H, w.I, w.fmt)
+            layers.append(layer.MoeLayer(w.E, w.H, w.I, w.k, w.fmt, gu, dn, A, B, w.lora_scale))
+
+        def args_of(l):
+            return (l.desc, T, x, lg, l.gate_up.codes, l.gate_up.scales, l.down.codes, l.down.scales, l.lora_A,
+                    l.lora_B, l.gu_bias, l.dn_bias, out, ws)
+
+        def graph_of(fn):
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.current_stream().wait_stream(side)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            return g
+
+        g_fwd = graph_of(lambda: [e4b.e4b_moe_forward(*args_of(l)) for l in layers])
+        g_gu = graph_of(lambda: [e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_GATE_UP, *args_of(l)) for l in layers])
+        g_dn = graph_of(lambda: [e4b.e4b_moe_forward_stage(e4b.E4B_STAGE_DOWN, *args_of(l)) for l in layers])
+
+        def per_layer_ms(g, n=None, sampler=None):
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            if n is None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                n = int(min(2000, max(5, target_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if sampler:
+                sampler.start()
+            e0.record()
+            for _ in range(n):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            clk = sampler.summary() if sampler else None
+            return max_over_ranks(e0.elapsed_time(e1) / (n * len(layers))), n, clk
+
+        ms, n, clk = per_layer_ms(g_fwd, sampler=ClockSampler(physical_gpu_index(dev.index or 0)))
+        gu_ms, _, _ = per_layer_ms(g_gu, n)
+        dn_ms, _, _ = per_layer_ms(g_dn, n)
+        if e4b.e4b_device_status(ws) != e4b.E4B_OK:
+            raise RuntimeError(f"device status reported an error in config {wname} T={T}")
+        active = max(min(R, w.E), 1)
+        avg = (R + active - 1) // active
+        rec = {"workload": wname, "T": T, "ms_per_step": ms, "tokens_per_s": T / (ms * 1e-3),
+               "bound": "tensor" if tensor else "hbm", "touched_experts": touched,
+               "kernel": "decode kernel (warp-level MMA)" if avg <= 12 else "tcgen05 tiles",
+               "timing": f"{n} graph replays of {len(layers)} layer cop{'y' if len(layers) == 1 else 'ies'} "
+                         f"(distinct weight addresses, {wbytes * len(layers) / 1e6:.0f} MB touched per replay)",
+               "clocks": clk}
+        if tensor:
+            rec["gate_up"] = {"ms": gu_ms, "flops": gu_flops, "tflops": gu_flops / (gu_ms * 1e-3) / 1e12}
+            rec["down"] = {"ms": dn_ms, "flops": dn_flops, "tflops": dn_flops / (dn_ms * 1e-3) / 1e12}
+            rec["layer_tflops"] = w.flops(T) / (ms * 1e-3) / 1e12
+            for kk in ("gate_up", "down"):
+                rec[kk]["frac"] = rec[kk]["tflops"] / peaks["bf16_tflops"]
+            rec["layer_frac"] = rec["layer_tflops"] / peaks["bf16_tflops"]
+        else:
+            rec["gate_up"] = {"ms": gu_ms, "bytes": gu_bytes, "gbs": gu_bytes / (gu_ms * 1e-3) / 1e9}
+            rec["down"] = {"ms": dn_ms, "bytes": dn_bytes, "gbs": dn_bytes / (dn_ms * 1e-3) / 1e9}
+            rec["layer_weight_gbs"] = wbytes / (ms * 1e-3) / 1e9
+            for kk in ("gate_up", "down"):
+                rec[kk]["frac"] = rec[kk]["gbs"] / peaks["hbm_gbs"]
+            rec["layer_frac"] = rec["layer_weight_gbs"] / peaks["hbm_gbs"]
+            rec["layer_tflops"] = w.flops(T) / (ms * 1e-3) / 1e12
+        rows.append(rec)
+        del g_fwd, g_gu, g_dn, layers, lay, ws
+        torch.cuda.synchronize()
+    built.clear()
+    torch.cuda.empty_cache()
+    return rows
 
 
 def init_dist():
@@ -395,6 +527,10 @@ def bench_e4b(args, world, rank, local):
         del xq, cq, aq, cd, sd, od
 
     peaks, peak_kind = load_peaks()
+    configs = []
+    if args.workload == WORKLOAD and not args.no_configs:
+        with torch.cuda.nvtx.range("every configuration"):
+            configs = bench_configs(dev, peaks, max_over_ranks)
     for f in formats.values():
         f["frac_of_hbm"] = f["gbs"] / peaks["hbm_gbs"]
     # the library's kernel choice (tokens_per_tile 0): the decode kernel at <= 12 rows per routed expert
@@ -435,6 +571,7 @@ def bench_e4b(args, world, rank, local):
                 "path": "layer.HostForward.run: pinned host inputs -> device -> forward -> pinned host output, "
                         "one CUDA graph replay and a synchronize per step"},
         "standalone_kernels": formats,
+        "configs": configs,
         "gpu_launches": K * KERNELS_PER_STEP,
         "clocks": clocks,
     }
@@ -459,6 +596,7 @@ def main():
     ap.add_argument("--impl", choices=["e4b", "reference"], default="e4b")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-formats", action="store_true", help="skip timing the standalone format kernels")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing every configuration of the metric")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=WORKLOAD,
                     help="synthetic layer to time (default: the headline decode workload)")
     ap.add_argument("--tokens", type=int, default=None, help="tokens per step (default: the workload's largest)")

@@ -581,7 +581,10 @@ static __device__ __align__(256) uint8_t g_route_scratch[kNoAllocScratchBytes];
 
 // Device addresses of g_route_scratch, looked up once per device.  In host
 // code the array's name is only a host-side handle: the address the kernels
-// need comes from cudaGetSymbolAddress with that device current.
+// need comes from cudaGetSymbolAddress with that device current.  The cached
+// address belongs to the device's current context: a cudaDeviceReset between
+// calls would leave it stale, so callers must not reset the device while
+// they use this entry point.
 uint8_t* g_route_scratch_addr[64] = {};
 std::mutex g_route_scratch_mu;
 
@@ -620,9 +623,11 @@ extern "C" e4b_status e4b_route_noalloc(const uint16_t* logits, int32_t T, int32
   const e4b_status st = route_scratch_address(&scratch);
   if (st != E4B_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's contents: the status word and the
-  // last-block counter must start at zero
-  if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return E4B_ERR_CUDA;
+  // The array keeps the previous call's contents.  The status word and the
+  // last-block counter must start at zero; launch_route clears them itself
+  // (inside the single routing block for T <= 128, else by a memset ahead of
+  // the multi-block kernels), and every other region is written before it is
+  // read, so nothing else needs clearing.
   RouteBuffers b;
   b.status = reinterpret_cast<int32_t*>(scratch);
   b.done_counter = reinterpret_cast<uint32_t*>(b.status + 2);

@@ -154,24 +154,25 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
     E, H, I = w.E, w.H, w.I
     if w.fmt == "mxfp4":
         lo, hi = w.exp_range
-        gc, gs = synth.stack_mxfp4(E, 2 * I, H, lo, hi, w.seed, "gate_up")
-        dc, ds = synth.stack_mxfp4(E, H, I, lo, hi, w.seed, "down")
+        if w.scales == "extreme":
+            gc, gs = synth.stack_mxfp4_extreme(E, 2 * I, H, w.seed, "gate_up", gate_rows=I)
+            dc, ds = synth.stack_mxfp4_extreme(E, H, I, w.seed, "down")
+        else:
+            gc, gs = synth.stack_mxfp4(E, 2 * I, H, lo, hi, w.seed, "gate_up")
+            dc, ds = synth.stack_mxfp4(E, H, I, lo, hi, w.seed, "down")
         gu = PackedStack(torch.from_numpy(gc).to(device), torch.from_numpy(gs).to(device), E, 2 * I, H, "mxfp4")
         dn = PackedStack(torch.from_numpy(dc).to(device), torch.from_numpy(ds).to(device), E, H, I, "mxfp4")
     else:
         gu = quantize_stack_nf4(torch.from_numpy(synth.stack_normal_f32(E, 2 * I, H, w.weight_std, w.seed,
-                                                                        "gate_up")).to(device))
+                                                                        "gate_up", w.zero_block_every)).to(device))
         dn = quantize_stack_nf4(torch.from_numpy(synth.stack_normal_f32(E, H, I, w.weight_std, w.seed,
-                                                                        "down")).to(device))
+                                                                        "down", w.zero_block_every)).to(device))
         if w.absmax_dq:   # the codes stay; the absmax is replaced by a synthetic nested-form one
             gu = PackedStack(gu.codes, nf4_dq_tensors(E, 2 * I * H // 64, w.seed, "gate_up_absmax", device),
                              E, 2 * I, H, "nf4_dq")
             dn = PackedStack(dn.codes, nf4_dq_tensors(E, H * I // 64, w.seed, "down_absmax", device),
                              E, H, I, "nf4_dq")
-    A = B = None
-    if w.lora_rank:
-        A = bits_tensor(synth.normal_bf16((E, H, w.lora_rank), 1.0 / w.lora_rank, w.seed, "lora_A"), device)
-        B = bits_tensor(synth.normal_bf16((E, w.lora_rank, 2 * I), 0.01, w.seed, "lora_B"), device)
+    A, B = synthetic_lora(w, device)
     bgu = bdn = None
     if w.bias_std > 0:
         bgu = torch.from_numpy(synth.normal_f32((E, 2 * I), w.bias_std, w.seed, "gate_up_bias")).to(device)
@@ -179,6 +180,15 @@ def synthetic_layer(w: Workload, device, tokens_per_tile=0):
     if w.interleaved:
         gu, bgu = deinterleave_gate_up(gu, bgu)
     return MoeLayer(E, H, I, w.k, gu.fmt, gu, dn, A, B, w.lora_scale, tokens_per_tile, bgu, bdn, w.glu, w.gating)
+
+
+def synthetic_lora(w: Workload, device):
+    """The workload's LoRA factors (A [E, H, r] ~ N(0, 1/r), B [E, r, 2I] ~ N(0, 0.01), bf16), or (None, None)."""
+    if not w.lora_rank:
+        return None, None
+    A = bits_tensor(synth.normal_bf16((w.E, w.H, w.lora_rank), 1.0 / w.lora_rank, w.seed, "lora_A"), device)
+    B = bits_tensor(synth.normal_bf16((w.E, w.lora_rank, 2 * w.I), 0.01, w.seed, "lora_B"), device)
+    return A, B
 
 
 def nf4_dq_tensors(E, n_per_expert, seed, name, device):

@@ -28,6 +28,8 @@ class Workload:
     interleaved: bool = False             # gate_up drawn with gate/up rows interleaved, de-interleaved at load
     gating: str = "topk"                  # router weights: "topk" (softmax over the picks) or "all"
     absmax_dq: bool = False               # NF4: absmax stored double-quantised (nested form)
+    zero_block_every: int = 0             # NF4: every n-th 64-value block of the fp32 weights is zero
+    scales: str = "uniform"               # MXFP4: "uniform" (exp_range) or "extreme" (synth.expert_mxfp4_extreme)
     seed: int = 0
     notes: str = field(default="", compare=False)
 

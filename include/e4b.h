@@ -229,11 +229,14 @@ e4b_status e4b_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, in
  *   Arguments and outputs are those of e4b_route, minus ws/ws_bytes.
  *   Scratch lives in one fixed 1 MiB device array inside the library; every
  *   GPU that loads the library holds it until the process exits.  Inputs that
- *   would need more (256 B + 128-token blocks x E x 4 B + T*k x 4 B, e.g. T
- *   above 16384 at E = 256, k = 8) return E4B_ERR_UNSUPPORTED; nothing runs.
+ *   would need more (256 B + ceil(T / 128) x E x 4 B + T*k x 4 B, each part
+ *   rounded up to 256 B; e.g. T above 26200 at E = 256, k = 8) return
+ *   E4B_ERR_UNSUPPORTED before anything is looked up or launched.
  *   It allocates nothing: no cudaMalloc, cudaFree or allocating routine.
  *   The first call on each device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   The address is kept for the process: do not reset the device
+ *   (cudaDeviceReset) between calls.
  *   Every call on a device shares the one array, so calls that overlap on the
  *   GPU (different streams, no ordering between them) race and corrupt each
  *   other's results: order them on one stream or with events.

@@ -33,6 +33,11 @@ Readings where the pages are silent:
   STORED transposed and K-contiguous, gate_up as [2I, H] and down as [H, I],
   so quantisation blocks run along the reduction dimension (the MX layout and
   the released gpt-oss blocks layout).
+* An MXFP4 weight is the exact bf16 decode of its code and scale ("Two
+  fidelity paths" on the MXFP4 page: the released bytes decode bit-exactly
+  into bf16).  For E8M0 bytes up to 252 that is the exact product; above, a
+  product beyond the bf16 range is +-inf, as in the standalone decode, and
+  byte 255 is NaN.  NF4 weights stay the exact fp64 product level * absmax.
 * The fused 2I output is [gate | up] halves, not interleaved (interleaving is
   named on the MXFP4 page as a gpt-oss peculiarity, outside the stock epilogue).
 * One LoRA adapter per expert on the fused gate_up output: A_e [H, r],
@@ -50,7 +55,7 @@ Readings where the pages are silent:
 """
 import numpy as np
 
-from .bf16 import bf16_bits_to_f64
+from .bf16 import bf16_bits_to_f64, round_to_bf16
 from .mxfp4 import decode_mxfp4
 from .nf4 import decode_nf4
 from .route import route_values
@@ -68,7 +73,7 @@ def decode_expert(fmt, codes, scales, e, rows, cols):
         return decode_nf4(c, s, per).reshape(rows, cols)
     if fmt == MXFP4:
         s = np.asarray(scales).reshape(-1)[e * per // 32:(e + 1) * per // 32]
-        return decode_mxfp4(c, s, per).reshape(rows, cols)
+        return round_to_bf16(decode_mxfp4(c, s, per)).reshape(rows, cols)
     raise ValueError(fmt)
 
 

@@ -40,6 +40,21 @@ def assert_close_layer(got, ref, what=""):
     return rel, mx
 
 
+def assert_close_layer_nonfinite(got, ref, what=""):
+    """As assert_close_layer for outputs that may hold NaN or +-inf: the oracle's value rounded to bf16
+    decides where they are, and the GPU output must be NaN, +inf and -inf at exactly those places; the
+    finite rest is held to the same bounds."""
+    from oracle.bf16 import round_to_bf16
+    got = np.asarray(got, np.float64)
+    refb = round_to_bf16(np.asarray(ref, np.float64))
+    assert np.array_equal(np.isnan(got), np.isnan(refb)), f"{what}: NaN positions differ"
+    assert np.array_equal(np.isposinf(got), np.isposinf(refb)), f"{what}: +inf positions differ"
+    assert np.array_equal(np.isneginf(got), np.isneginf(refb)), f"{what}: -inf positions differ"
+    fin = np.isfinite(refb)
+    assert fin.sum() > fin.size // 4, f"{what}: too few finite outputs to compare"
+    return assert_close_layer(got[fin], np.asarray(ref, np.float64)[fin], what)
+
+
 def touched_experts(logits_bits, k):
     r = oroute.route(logits_bits, k)
     return sorted(set(r["ids"].reshape(-1).tolist()))
@@ -55,16 +70,22 @@ def oracle_stacks(w, experts):
         dc = np.zeros((E, H * I // 2), np.uint8)
         ds = np.zeros((E, H * I // 32), np.uint8)
         for e in experts:
-            gc[e], gs[e] = synth.expert_mxfp4(e, 2 * I, H, lo, hi, w.seed, "gate_up")
-            dc[e], ds[e] = synth.expert_mxfp4(e, H, I, lo, hi, w.seed, "down")
+            if w.scales == "extreme":
+                gc[e], gs[e] = synth.expert_mxfp4_extreme(e, 2 * I, H, w.seed, "gate_up", gate_rows=I)
+                dc[e], ds[e] = synth.expert_mxfp4_extreme(e, H, I, w.seed, "down")
+            else:
+                gc[e], gs[e] = synth.expert_mxfp4(e, 2 * I, H, lo, hi, w.seed, "gate_up")
+                dc[e], ds[e] = synth.expert_mxfp4(e, H, I, lo, hi, w.seed, "down")
     else:
         gc = np.zeros((E, 2 * I * H // 2), np.uint8)
         gs = np.zeros((E, 2 * I * H // 64), np.float32)
         dc = np.zeros((E, H * I // 2), np.uint8)
         ds = np.zeros((E, H * I // 64), np.float32)
         for e in experts:
-            gc[e], gs[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, 2 * I, H, w.weight_std, w.seed, "gate_up"))
-            dc[e], ds[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, H, I, w.weight_std, w.seed, "down"))
+            gc[e], gs[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, 2 * I, H, w.weight_std, w.seed, "gate_up",
+                                                                     w.zero_block_every))
+            dc[e], ds[e] = onf4.quantize_nf4(synth.expert_normal_f32(e, H, I, w.weight_std, w.seed, "down",
+                                                                     w.zero_block_every))
         if w.absmax_dq:   # the stored absmax is the nested form's expansion
             gs = onf4.expand_absmax_dq(*synth.nf4_dq_absmax(E, 2 * I * H // 64, w.seed, "gate_up_absmax"))
             ds = onf4.expand_absmax_dq(*synth.nf4_dq_absmax(E, H * I // 64, w.seed, "down_absmax"))
@@ -109,7 +130,8 @@ def oracle_epilogue(w):
     return bgu, bdn
 
 
-def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=0, x=None, logits=None):
+def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=0, x=None, logits=None,
+                    nonfinite=False):
     """Runs the GPU forward on all T tokens and compares `sample` rows (default all) with the oracle."""
     dev = device()
     if x is None:
@@ -133,4 +155,5 @@ def run_and_compare(w, T, tokens_per_tile=0, sample=None, lay=None, seed_offset=
                               lora_A_bits=A, lora_B_bits=B, lora_scale=w.lora_scale, gu_bias=bgu, dn_bias=bdn,
                               glu=w.glu, gating=w.gating)
     got = bf16_to_f64(out)[rows]
-    return assert_close_layer(got, ref, f"{w.name} T={T} tile={tokens_per_tile}"), lay, out
+    check = assert_close_layer_nonfinite if nonfinite else assert_close_layer
+    return check(got, ref, f"{w.name} T={T} tile={tokens_per_tile}"), lay, out

@@ -53,6 +53,11 @@ def test_route_validation(L):
     # an unknown gating mode is refused before anything else is looked at
     assert L.e4b_route(None, 4, 8, 2, 2, None, None, 256, None, 256, 1 << 20, None) == e4b.E4B_ERR_INVALID_ARG
     assert L.e4b_route_noalloc(None, 4, 8, 2, -1, None, None, 256, None, None) == e4b.E4B_ERR_INVALID_ARG
+    # the fixed scratch of the no-alloc entry takes T = 26200 at E = 256, k = 8 and refuses one more
+    # token before anything is looked up or launched (no GPU is touched here)
+    fake = 4096
+    assert L.e4b_route_noalloc(fake, 26201, 256, 8, 0, fake, fake, fake, fake, None) == e4b.E4B_ERR_UNSUPPORTED
+    assert L.e4b_route_noalloc(fake, 10 ** 6, 8, 2, 0, fake, fake, fake, fake, None) == e4b.E4B_ERR_UNSUPPORTED
     assert L.e4b_route_workspace_bytes(16, 8, 2) > 0
     assert L.e4b_route_workspace_bytes(16, 8, 9) == 0
 

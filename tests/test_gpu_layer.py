@@ -87,9 +87,30 @@ def test_lora_tiny_and_zero_b(fmt, tpt):
 
 
 @pytest.mark.parametrize("tpt", [0, 32])
-@pytest.mark.parametrize("T", [1, 8])
+@pytest.mark.parametrize("T", [1, 8, 32])
 def test_qwen3_nf4_decode_full(T, tpt):
     run_and_compare(QWEN, T, tokens_per_tile=tpt)
+
+
+# ---------------------------------------------------------------- format edge cases inside the forward
+
+@pytest.mark.parametrize("tpt", [0, 8, 32, 256])
+def test_mxfp4_extreme_scales_layer(tpt):
+    # E8M0 bytes at both ends of the range through either GEMM kernel's dequant: gate rows scaled by
+    # 2^-127 .. 2^-121 (byte 0 is a bf16-subnormal scale), down rows by 2^113 .. 2^125, a sprinkling of
+    # down blocks at 253 / 254 (products beyond bf16: +-inf weights) and 255 (NaN), and a NaN up block
+    # in expert 0.  NaN and +-inf must land exactly where the oracle puts them.
+    w = Workload("extreme", "mxfp4", E=6, H=320, I=192, k=2, tokens=(100,), scales="extreme", seed=31)
+    run_and_compare(w, 100, tokens_per_tile=tpt, nonfinite=True)
+
+
+@pytest.mark.parametrize("tpt", [0, 8, 32, 256])
+def test_nf4_zero_blocks_layer(tpt):
+    # every 5th 64-value block of both stacks is zero: absmax 0, code 7 everywhere in it
+    w = Workload("zero_blocks", "nf4", E=6, H=320, I=192, k=2, tokens=(100,), zero_block_every=5, seed=32)
+    (_, _), lay, _ = run_and_compare(w, 100, tokens_per_tile=tpt)
+    absmax = lay.gate_up.scales.view(w.E, -1).cpu().numpy()
+    assert np.all(absmax[:, 4::5] == 0) and np.all(absmax[:, 0::5] > 0)
 
 
 @pytest.mark.parametrize("tpt", [0, 8, 32])

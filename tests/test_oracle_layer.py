@@ -323,3 +323,45 @@ def test_deinterleave_restores_released_gate_up_tensors(fmt):
     assert np.array_equal(moe.deinterleave_rows(ic, E, I), codes)
     assert np.array_equal(moe.deinterleave_rows(isc, E, I), scales)
     assert np.array_equal(moe.deinterleave_rows(ib, E, I), bgu)
+
+
+# ---------------------------------------------------------------- MXFP4 weights at the ends of the E8M0 range
+
+def test_layer_mxfp4_weights_are_the_bf16_decode_for_every_code_and_scale():
+    # the layer decodes every (code byte, scale byte) pair to the standalone bf16 decode, which is
+    # pinned exhaustively against float products (test_oracle_formats); rows of 64 values, one per scale
+    codes = np.repeat(np.arange(256, dtype=np.uint8)[None, :], 256, axis=0).reshape(-1)   # [scale][code]
+    scales = np.repeat(np.arange(256, dtype=np.uint8), 16)                                 # 512 values per scale
+    n = codes.size * 2
+    got = moe.decode_expert("mxfp4", codes, scales, 0, 256, 512).reshape(-1)
+    ref = bf16.bf16_bits_to_f64(mxfp4.dequant_mxfp4_bf16(codes, scales, n))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin])
+    assert np.isposinf(got).sum() > 0 and np.isneginf(got).sum() > 0    # bytes 253 and 254 overflow
+    assert np.all(np.isfinite(got[: 253 * 512]))                         # bytes up to 252 never do
+
+
+def test_forward_nan_and_overflowing_down_scales_reach_their_output_columns_only():
+    E, H, I, T = 1, 64, 64, 6
+    gu = synth.stack_mxfp4(E, 2 * I, H, -4, 2, 7, "gu")
+    dc, ds = synth.stack_mxfp4(E, H, I, -4, 2, 7, "dn")
+    dc, ds = dc.copy().reshape(H, I // 2), ds.copy().reshape(H, I // 32)
+    ds[3, 0] = 255                      # row 3, first block: NaN scale
+    ds[5, 1] = 254                      # row 5, second block: 2^127 ...
+    dc[5, 16:32] = 0                    # ... all codes zero but element 32 + 7 = code 4 (2.0): +inf
+    dc[5, 16 + 3] = 0x40
+    ds[7, :] = 252                      # row 7: largest scale whose products stay finite
+    dc[7, :] = 0x66                     # codes 6 (4.0): 4 * 2^125
+    x = synth.normal_bf16((T, H), 1.0, 7, "x")
+    logits = synth.normal_bf16((T, E), 1.0, 7, "logits")
+    out, _ = moe.moe_forward(x, logits, 1, "mxfp4", E, H, I, gu[0], gu[1], dc.reshape(-1), ds.reshape(-1))
+    X = bf16.bf16_bits_to_f64(x)
+    Wg = mxfp4.decode_mxfp4(gu[0], gu[1], 2 * I * H).reshape(2 * I, H)
+    gate, up = X @ Wg[:I].T, X @ Wg[I:].T
+    h = gate / (1.0 + np.exp(-gate)) * up                                   # textbook SwiGLU, [T, I]
+    assert np.all(np.isnan(out[:, 3]))
+    assert np.array_equal(out[:, 5], np.copysign(np.inf, h[:, 39]))        # element 39 = 32 + 7
+    assert np.allclose(out[:, 7], h.sum(axis=1) * 4.0 * 2.0 ** 125, rtol=1e-12)
+    others = np.setdiff1d(np.arange(H), [3, 5])
+    assert np.all(np.isfinite(out[:, others]))
