@@ -28,6 +28,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// The forward's kernels are launched with programmatic stream serialization:
+// a kernel may start while the one before it on the stream is still running.
+// Each does its independent set-up (barriers, byte tables, tensor-map
+// prefetch) first, then pdl_wait(), which returns once every earlier grid on
+// the stream has completed and its memory is visible; nothing written by an
+// earlier kernel is read, and nothing an earlier kernel may still read is
+// written, before it.  pdl_launch_dependents() lets the next kernel start its
+// own set-up.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

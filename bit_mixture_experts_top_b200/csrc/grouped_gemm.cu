@@ -279,14 +279,18 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       lut[i] = *reinterpret_cast<uint32_t*>(&v);
     }
   }
-  for (int i = threadIdx.x; i <= p.E; i += C::THREADS) {
-    s_chunk[i] = __ldg(p.chunk_off + i);
-    s_off[i] = __ldg(p.expert_offsets + i);
-  }
   if (warp == WARP_RAW && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_act);
     if (MODE == 0 && p.lora_rank > 0) tma_prefetch_desc(&tm_xa);
+  }
+  // the set-up above depends on nothing an earlier kernel writes; the tile tables,
+  // activations and tensor memory (held by an earlier grid until it ends) below do
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= p.E; i += C::THREADS) {
+    s_chunk[i] = __ldg(p.chunk_off + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
   }
   if (warp == WARP_MMA) {
     tmem_alloc(s_tmem, C::TMEM_COLS);
@@ -696,8 +700,9 @@ e4b_status launch_typed(const GroupedGemmLaunch& g, const CUtensorMap& tc, const
   const int64_t max_tiles = (active + (g.R + BN - 1) / BN) * prm.n_blocks;
   const int64_t sms = device_sm_count();
   const int grid = static_cast<int>(max_tiles < sms ? (max_tiles > 0 ? max_tiles : 1) : sms);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tc, ta, tx, prm);
-  return cudaGetLastError() == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, tc, ta, tx, prm) == cudaSuccess
+             ? E4B_OK
+             : E4B_ERR_CUDA;
 }
 
 template <int BN>

@@ -111,6 +111,8 @@ __global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __r
                                                               int32_t* __restrict__ sorted_slot,
                                                               int32_t* __restrict__ slot_pos) {
   __shared__ int32_t s_wc[kWarps][kMaxExperts];
+  pdl_wait();
+  pdl_launch_dependents();
   rank_block<kWarps>(blockIdx.x, topk_ids, T, E, k, block_base, sorted_slot, slot_pos, s_wc);
 }
 
@@ -126,6 +128,8 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
   __shared__ int32_t s_tot[kMaxExperts + 1];
   __shared__ bool s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   for (int e = tid; e < E; e += kTopkThreads) s_cnt[e] = 0;
   __syncthreads();
 
@@ -249,11 +253,15 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
   }
 }
 
-// T <= 128 (one routing block): top-k, histogram, scans and the stable rank in
-// one block with every intermediate in shared memory, no cross-block protocol.
-// The block also zeroes the status words of the workspace first (the caller
-// skips its memset), so a small forward starts with a single launch.
-__global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
+// T <= 4 * NW (one routing block of NW warps, 4 tokens per warp): top-k,
+// histogram, scans and the stable rank in one block with every intermediate in
+// shared memory, no cross-block protocol.  The block also zeroes the status
+// words of the workspace first (the caller skips its memset), so a small
+// forward starts with a single launch.  Decode batches (T <= 32) take an
+// 8-warp block, whose barriers and shared-memory clears cost a quarter of the
+// 32-warp block's.
+template <int NW>
+__global__ void __launch_bounds__(NW * 32) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
                                                                   int k, int gating, int tokens_per_tile,
                                                                   int32_t* status_words,
                                                                   int32_t* __restrict__ topk_ids,
@@ -263,20 +271,23 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
                                                                   int32_t* __restrict__ sorted_slot,
                                                                   int32_t* __restrict__ slot_pos) {
   __shared__ int16_t s_ids[kRouteTokensPerBlock * kMaxTopK];
-  __shared__ __align__(16) int16_t s_wc[kTopkWarps][kMaxExperts];   // per-warp counts, then running positions
+  constexpr int kW = NW, kT = NW * 32;
+  __shared__ __align__(16) int16_t s_wc[kW][kMaxExperts];   // per-warp counts, then running positions
   __shared__ int32_t s_cnt[kMaxExperts];
   __shared__ int32_t s_off[kMaxExperts];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   if (status_words && tid < kStatusBytes / 4) status_words[tid] = 0;
-  for (int e = tid; e < kMaxExperts; e += kTopkThreads) s_cnt[e] = 0;
-  for (int i = tid; i < kTopkWarps * kMaxExperts; i += kTopkThreads) (&s_wc[0][0])[i] = 0;
+  for (int e = tid; e < kMaxExperts; e += kT) s_cnt[e] = 0;
+  for (int i = tid; i < kW * kMaxExperts; i += kT) (&s_wc[0][0])[i] = 0;
   __syncthreads();
 
   const int per_lane = (E + 31) >> 5;
   uint32_t key[kTokPerWarp][kMaxExperts / 32];
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
-    const int t = warp + kTopkWarps * q;
+    const int t = warp + kW * q;
     const uint16_t* row = logits + static_cast<int64_t>(t) * E;
 #pragma unroll
     for (int j = 0; j < kMaxExperts / 32; ++j) {
@@ -286,7 +297,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
   }
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
-    const int t = warp + kTopkWarps * q;
+    const int t = warp + kW * q;
     if (t >= T) break;
     uint32_t mine = 0;
     float all_sum = 0.0f;
@@ -358,7 +369,7 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
   }
   // stable rank: warp w owns the contiguous slot segment [w0, w1)
   const int n = T * k;
-  const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+  const int seg = ((n + kW - 1) / kW + 31) / 32 * 32;
   const int w0 = warp * seg, w1 = min(n, w0 + seg);
   for (int s = w0 + lane; s < w1; s += 32) {
     const int id = s_ids[s];
@@ -366,9 +377,9 @@ __global__ void __launch_bounds__(kTopkThreads) route_small_kernel(const uint16_
     atomicAdd(reinterpret_cast<int*>(&s_wc[warp][id & ~1]), 1 << (16 * (id & 1)));
   }
   __syncthreads();
-  for (int e = tid; e < E; e += kTopkThreads) {
+  for (int e = tid; e < E; e += kT) {
     int32_t run = s_off[e];
-    for (int w = 0; w < kTopkWarps; ++w) {
+    for (int w = 0; w < kW; ++w) {
       const int32_t c = s_wc[w][e];
       s_wc[w][e] = static_cast<int16_t>(run);
       run += c;
@@ -403,6 +414,8 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __rest
                                                           const uint16_t* __restrict__ lora_A, int rank,
                                                           float scale, uint16_t* __restrict__ xa) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t r = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   if (r >= R) return;
   const int32_t slot = sorted_slot[r];
@@ -481,6 +494,8 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
                                                            const float* __restrict__ topk_w,
                                                            const int32_t* __restrict__ slot_pos, int k, int H,
                                                            uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t t = blockIdx.x;
   const int c = blockIdx.y * kThreads + threadIdx.x;
   if (c >= H / 4) return;
@@ -524,19 +539,21 @@ cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k
   }
   const int nblk = route_blocks(T);
   if (nblk == 1) {
-    route_small_kernel<<<1, kTopkThreads, 0, s>>>(logits, T, E, k, gating, tokens_per_tile, status_words, b.topk_ids,
-                                                  b.topk_w, b.expert_offsets, b.chunk_off, b.sorted_slot,
-                                                  b.slot_pos);
-    return cudaGetLastError();
+    if (T <= 4 * 8)
+      return launch_pdl(route_small_kernel<8>, dim3(1), dim3(8 * 32), 0, s, logits, T, E, k, gating,
+                        tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
+                        b.sorted_slot, b.slot_pos);
+    return launch_pdl(route_small_kernel<kTopkWarps>, dim3(1), dim3(kTopkThreads), 0, s, logits, T, E, k, gating,
+                      tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
+                      b.sorted_slot, b.slot_pos);
   }
   if (status_words && cudaMemsetAsync(status_words, 0, kStatusBytes, s) != cudaSuccess) return cudaGetLastError();
-  route_topk_kernel<<<nblk, kTopkThreads, 0, s>>>(logits, T, E, k, gating, tokens_per_tile, nblk, b.topk_ids, b.topk_w,
-                                               b.block_counts, b.done_counter, b.expert_offsets, b.chunk_off,
-                                               b.sorted_slot, b.slot_pos);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(route_topk_kernel, dim3(nblk), dim3(kTopkThreads), 0, s, logits, T, E, k, gating,
+                               tokens_per_tile, nblk, b.topk_ids, b.topk_w, b.block_counts, b.done_counter,
+                               b.expert_offsets, b.chunk_off, b.sorted_slot, b.slot_pos);
   if (err != cudaSuccess || nblk == 1) return err;
-  route_rank_kernel<<<nblk, kThreads, 0, s>>>(b.topk_ids, T, E, k, b.block_counts, b.sorted_slot, b.slot_pos);
-  return cudaGetLastError();
+  return launch_pdl(route_rank_kernel, dim3(nblk), dim3(kThreads), 0, s, b.topk_ids, T, E, k,
+                    static_cast<const int32_t*>(b.block_counts), b.sorted_slot, b.slot_pos);
 }
 
 cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, const int32_t* sorted_slot,
@@ -545,17 +562,15 @@ cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, co
   (void)E;
   if (R == 0) return cudaSuccess;
   const int grid = (R + kWarps - 1) / kWarps;
-  gather_kernel<<<grid, kThreads, 0, s>>>(x, H, k, R, sorted_slot, topk_ids, x_sorted, lora_A, lora_rank,
-                                          lora_scale, xa);
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, dim3(grid), dim3(kThreads), 0, s, x, H, k, R, sorted_slot, topk_ids, x_sorted,
+                    lora_A, lora_rank, lora_scale, xa);
 }
 
 cudaError_t launch_combine(const float* y, const float* topk_w, const int32_t* slot_pos, int32_t T, int32_t k,
                            int32_t H, uint16_t* out, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const dim3 grid(T, (H / 4 + kThreads - 1) / kThreads);
-  combine_kernel<<<grid, kThreads, 0, s>>>(y, topk_w, slot_pos, k, H, out);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(kThreads), 0, s, y, topk_w, slot_pos, k, H, out);
 }
 
 }  // namespace e4b

@@ -277,10 +277,6 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   }
   if (FMT == E4B_NF4 && threadIdx.x < 16)
     s_level[threadIdx.x] = static_cast<uint16_t>(p.level2[threadIdx.x >> 1] >> (16 * (threadIdx.x & 1)));
-  for (int i = threadIdx.x; i <= p.E; i += SK_THREADS) {
-    s_chunk[i] = __ldg(p.chunk_off + i);
-    s_off[i] = __ldg(p.expert_offsets + i);
-  }
   if (warp == SK_PRODUCER && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     tma_prefetch_desc(&tm_x);
@@ -300,6 +296,14 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
     }
     lut[at] = v;
   }
+  // everything above depends on nothing an earlier kernel writes; the unit
+  // tables, activations and counters below do
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i <= p.E; i += SK_THREADS) {
+    s_chunk[i] = __ldg(p.chunk_off + i);
+    s_off[i] = __ldg(p.expert_offsets + i);
+  }
   __syncthreads();
 
   const WaitCtx wctx{s_abort, p.status, p.wait_limit_ns};
@@ -310,13 +314,11 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
   if (warp == SK_PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      bool drained = false;
-      auto fetch = [&]() {
-        if (drained) return total;
-        const int u = static_cast<int>(atomicAdd(&p.counters[0], 1u));
-        if (u >= total) drained = true;
-        return u < total ? u : total;
-      };
+      // Unit blockIdx.x first (no atomic ahead of the first copy), then units
+      // gridDim.x + 0, 1, ... in the order CTAs ask for them.  A fetched index is
+      // compared with `total` only where it is used, so the atomic's round trip
+      // overlaps the copies issued before that point; an index >= total ends the CTA.
+      auto fetch = [&]() { return static_cast<int>(gridDim.x + atomicAdd(&p.counters[0], 1u)); };
       uint32_t armed = 0, par = 0, sarmed = 0, spar = 0;
       bool ok = true;
       // unit k's scale rows go to buffer k % SK_SBUF, one unit ahead of its stages
@@ -350,7 +352,8 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         spar = (spar & ~(1u << sb)) | (sph << sb);
         return true;
       };
-      int q0 = fetch(), q1 = fetch(), q2 = fetch();
+      const int q0 = static_cast<int>(blockIdx.x);
+      int q1 = q0 < total ? fetch() : total, q2 = total;
       int slot = 0;
       uint32_t ph = 0;
       int u = q0;
@@ -374,12 +377,12 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           if (++slot == p.stages) { slot = 0; ph ^= 1u; }
         }
         if (!ok) break;
+        if (k == 0) q2 = fetch();     // the second request goes out once the first unit's copies are issued
         u = q1;
         q1 = q2;
-        q2 = fetch();
+        q2 = u < total ? fetch() : total;
         ok = issue_scales(k + 1, u);
       }
-      while (!drained) (void)fetch();
       // the last CTA through resets the counters for the next launch
       __threadfence();
       if (atomicAdd(&p.counters[1], 1u) == gridDim.x - 1) {
@@ -602,8 +605,9 @@ e4b_status launch_typed(const CUtensorMap& tc, const CUtensorMap& tx, const CUte
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SK_SMEM_LIMIT);
   });
   if (attr_err != cudaSuccess) return E4B_ERR_CUDA;
-  kern<<<device_sm_count(), SK_THREADS, smem, s>>>(tc, tx, ts, prm);
-  return cudaGetLastError() == cudaSuccess ? E4B_OK : E4B_ERR_CUDA;
+  return launch_pdl(kern, dim3(device_sm_count()), dim3(SK_THREADS), smem, s, tc, tx, ts, prm) == cudaSuccess
+             ? E4B_OK
+             : E4B_ERR_CUDA;
 }
 
 int scale_row_bytes(int32_t K, int32_t fmt) { return fmt == E4B_NF4 ? K / 16 : K / 32; }
