@@ -129,5 +129,9 @@ int device_sm_count();
 // driver entry point; false when the driver refuses the description.
 bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+// 3-D tiled tensor map: dims d0 (contiguous), d1 (stride1_bytes apart), d2 (stride2_bytes apart).
+bool encode_tma_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0, uint64_t d1,
+                   uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2,
+                   CUtensorMapSwizzle swz);
 
 }  // namespace e4b

@@ -367,11 +367,16 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
           if (!mbar_wait(&empty[slot], ph ^ 1u, wctx, 712)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[slot], STAGE_BYTES);
           uint8_t* dst = ring + slot * STAGE_BYTES;
-          tma_load_2d(dst, &tm_codes, &full[slot], SK_KST / 2 * st, ya);
-          tma_load_2d(dst + SK_CODE_BYTES / 2, &tm_codes, &full[slot], SK_KST / 2 * st, yb);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tma_load_2d(dst + SK_CODE_BYTES + 1024 * TG * i, &tm_x, &full[slot], SK_KST * st + 64 * i, un.t0);
+          // Two copies per stage (the copy engine's throughput per SM, about 23 bytes per
+          // clock plus a fixed cost per copy instruction, bounds the stream): the codes of
+          // both 64-row halves of the unit (gate and up rows through the view
+          // [expert x half][row][K], or 128 consecutive rows), and the chunk's activation
+          // rows of the stage's four 64-K blocks (view [block][row][64 K]).
+          if (MODE == 0)
+            tma_load_3d(dst, &tm_codes, &full[slot], SK_KST / 2 * st, 64 * un.nb, 2 * un.e);
+          else
+            tma_load_2d(dst, &tm_codes, &full[slot], SK_KST / 2 * st, ya);
+          tma_load_3d(dst + SK_CODE_BYTES, &tm_x, &full[slot], 0, un.t0, 4 * st);
           armed |= 1u << slot;
           par = (par & ~(1u << slot)) | (ph << slot);
           if (++slot == p.stages) { slot = 0; ph ^= 1u; }
@@ -672,11 +677,18 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   }
   CUtensorMap tc, tx, ts;
   const uint64_t code_rows = static_cast<uint64_t>(g.E) * g.N;
-  if (!encode_tma_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2, SK_KST / 2, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-    return E4B_ERR_CUDA;
-  if (!encode_tma_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, g.K, g.R, static_cast<uint64_t>(g.K) * 2, 64,
-                     tok, CU_TENSOR_MAP_SWIZZLE_128B))
+  const bool coded = g.mode == 0
+                         // gate_up: [E x {gate, up}] x I rows x K/2 bytes; one box holds both 64-row halves
+                         ? encode_tma_3d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, g.I,
+                                         2 * static_cast<uint64_t>(g.E), g.K / 2,
+                                         static_cast<uint64_t>(g.I) * (g.K / 2), SK_KST / 2, 64, 2,
+                                         CU_TENSOR_MAP_SWIZZLE_128B)
+                         : encode_tma_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.codes, g.K / 2, code_rows, g.K / 2,
+                                         SK_KST / 2, SK_ROWS, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!coded) return E4B_ERR_CUDA;
+  // activations [R, K] viewed as [K / 64 blocks][R rows][64 K]: one box = the stage's four blocks
+  if (!encode_tma_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.act, 64, g.R, g.K / 64, static_cast<uint64_t>(g.K) * 2,
+                     128, 64, tok, 4, CU_TENSOR_MAP_SWIZZLE_128B))
     return E4B_ERR_CUDA;
   if (prm.scale_tma) {
     const CUtensorMapSwizzle sw = prm.srow == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
