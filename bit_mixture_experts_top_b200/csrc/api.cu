@@ -88,6 +88,32 @@ ForwardLayout forward_layout(const e4b_moe_desc& d, int32_t T) {
   return L;
 }
 
+// The training workspace: the forward's layout, then what the backward needs
+// besides it (the saved pre-activation G) and its own scratch.
+struct TrainLayout {
+  ForwardLayout fwd;
+  size_t g, dY, dG, dxa, dX, total;
+};
+
+TrainLayout train_layout(const e4b_moe_desc& d, int32_t T) {
+  TrainLayout L;
+  L.fwd = forward_layout(d, T);
+  const size_t R = static_cast<size_t>(T) * d.k;
+  size_t o = L.fwd.total;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += align_up(bytes);
+    return at;
+  };
+  L.g = take(R * 2 * d.I * 4);
+  L.dY = take(R * d.H * 2);
+  L.dG = take(R * 2 * d.I * 2);
+  L.dxa = take(d.lora_rank > 0 ? R * 16 * 4 : 0);
+  L.dX = take(R * d.H * 4);
+  L.total = o;
+  return L;
+}
+
 struct RouteLayout {
   size_t status, block_counts, slot_pos, total;
 };
@@ -297,7 +323,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
                              const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
                              const uint8_t* dn_codes, const void* dn_scales, const uint16_t* lora_A,
                              const uint16_t* lora_B, const float* gu_bias, const float* dn_bias, uint16_t* out,
-                             void* ws, size_t ws_bytes, e4b_stream stream) {
+                             void* ws, size_t ws_bytes, e4b_stream stream, bool train = false) {
   const e4b_status v = validate_desc(d, T);
   if (v != E4B_OK) return v;
   if (first < E4B_STAGE_ROUTE || last > E4B_STAGE_COMBINE || first > last) return E4B_ERR_INVALID_ARG;
@@ -305,7 +331,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   if ((lora_A != nullptr) != lora || (lora_B != nullptr) != lora) return E4B_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, kAlign)) return E4B_ERR_INVALID_ARG;
   const ForwardLayout L = forward_layout(*d, T);
-  if (ws_bytes < L.total) return E4B_ERR_INVALID_ARG;
+  if (ws_bytes < (train ? train_layout(*d, T).total : L.total)) return E4B_ERR_INVALID_ARG;
   const bool dq = d->format == E4B_NF4_DQ;
   if (T > 0) {
     if (!x || !logits || !gu_codes || !gu_scales || !dn_codes || !dn_scales || !out) return E4B_ERR_INVALID_ARG;
@@ -354,6 +380,8 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
   g.glu_alpha = d->glu_alpha;
   g.glu_limit = d->glu_limit;
   g.glu_beta = d->glu_beta;
+  g.g_out = nullptr;
+  float* g_keep = train ? at<float>(ws, train_layout(*d, T).g) : nullptr;
 
   for (int32_t stage = first; stage <= last; ++stage) {
     switch (stage) {
@@ -388,6 +416,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_rank = d->lora_rank;
         g.bias = gu_bias;
         g.out = h;
+        g.g_out = g_keep;
         const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
@@ -404,6 +433,7 @@ static e4b_status run_stages(int32_t first, int32_t last, const e4b_moe_desc* d,
         g.lora_rank = 0;
         g.bias = dn_bias;
         g.out = y;
+        g.g_out = nullptr;
         const e4b_status st = kc.decode ? launch_skinny_gemm(g, s) : launch_grouped_gemm(g, s);
         if (st != E4B_OK) return st;
         break;
@@ -432,6 +462,86 @@ e4b_status e4b_moe_forward_stage(int32_t stage, const e4b_moe_desc* d, int32_t T
                                  void* ws, size_t ws_bytes, e4b_stream stream) {
   return run_stages(stage, stage, d, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias,
                     dn_bias, out, ws, ws_bytes, stream);
+}
+
+size_t e4b_moe_train_workspace_bytes(const e4b_moe_desc* d, int32_t T) {
+  if (validate_desc(d, T) != E4B_OK) return 0;
+  return train_layout(*d, T).total;
+}
+
+e4b_status e4b_moe_forward_train(const e4b_moe_desc* d, int32_t T, const uint16_t* x, const uint16_t* logits,
+                                 const uint8_t* gu_codes, const void* gu_scales, const uint8_t* dn_codes,
+                                 const void* dn_scales, const uint16_t* lora_A, const uint16_t* lora_B,
+                                 const float* gu_bias, const float* dn_bias, uint16_t* out, void* ws,
+                                 size_t ws_bytes, e4b_stream stream) {
+  return run_stages(E4B_STAGE_ROUTE, E4B_STAGE_COMBINE, d, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales,
+                    lora_A, lora_B, gu_bias, dn_bias, out, ws, ws_bytes, stream, true);
+}
+
+e4b_status e4b_moe_backward(const e4b_moe_desc* d, int32_t T, const uint16_t* logits, const uint16_t* dout,
+                            const uint8_t* gu_codes, const void* gu_scales, const uint8_t* dn_codes,
+                            const void* dn_scales, const uint16_t* lora_A, const uint16_t* lora_B, float* dx,
+                            float* dlogits, float* dA, float* dB, void* ws, size_t ws_bytes, e4b_stream stream) {
+  const e4b_status v = validate_desc(d, T);
+  if (v != E4B_OK) return v;
+  const bool lora = d->lora_rank > 0;
+  if ((lora_A != nullptr) != lora || (lora_B != nullptr) != lora || (dA != nullptr) != lora ||
+      (dB != nullptr) != lora)
+    return E4B_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, kAlign)) return E4B_ERR_INVALID_ARG;
+  const TrainLayout L = train_layout(*d, T);
+  if (ws_bytes < L.total) return E4B_ERR_INVALID_ARG;
+  const bool dq = d->format == E4B_NF4_DQ;
+  if (T > 0) {
+    if (!logits || !dout || !gu_codes || !gu_scales || !dn_codes || !dn_scales || !dx || !dlogits)
+      return E4B_ERR_INVALID_ARG;
+    if (!aligned(dout, 4) || !aligned(dx, 16) || !aligned(dlogits, 4) || !aligned(gu_codes, 16) ||
+        !aligned(dn_codes, 16))
+      return E4B_ERR_INVALID_ARG;
+    if (dq ? !(valid_dq(static_cast<const e4b_nf4_dq*>(gu_scales)) && valid_dq(static_cast<const e4b_nf4_dq*>(dn_scales)))
+           : !(aligned(gu_scales, 16) && aligned(dn_scales, 16)))
+      return E4B_ERR_INVALID_ARG;
+    if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 2) || !aligned(dA, 4) || !aligned(dB, 4)))
+      return E4B_ERR_INVALID_ARG;
+  }
+  BackwardLaunch b;
+  b.T = T;
+  b.k = d->k;
+  b.E = d->E;
+  b.H = d->H;
+  b.I = d->I;
+  b.fmt = gemm_format(d->format);
+  b.gating = d->gating;
+  b.lora_rank = d->lora_rank;
+  b.lora_scale = d->lora_scale;
+  b.ep = Epilogue{nullptr, d->act, d->glu_alpha, d->glu_limit, d->glu_beta};
+  b.logits = logits;
+  b.dout = dout;
+  b.y = at<float>(ws, L.fwd.y);
+  b.topk_w = at<float>(ws, L.fwd.topk_w);
+  b.topk_ids = at<int32_t>(ws, L.fwd.topk_ids);
+  b.slot_pos = at<int32_t>(ws, L.fwd.slot_pos);
+  b.sorted_slot = at<int32_t>(ws, L.fwd.sorted_slot);
+  b.expert_offsets = at<int32_t>(ws, L.fwd.offsets);
+  b.x_sorted = at<uint16_t>(ws, L.fwd.x_sorted);
+  b.xa = lora ? at<uint16_t>(ws, L.fwd.xa) : nullptr;
+  b.G = at<float>(ws, L.g);
+  b.dY = at<uint16_t>(ws, L.dY);
+  b.dG = at<uint16_t>(ws, L.dG);
+  b.dxa = lora ? at<float>(ws, L.dxa) : nullptr;
+  b.dX = at<float>(ws, L.dX);
+  b.dx = dx;
+  b.dlogits = dlogits;
+  b.dA = dA;
+  b.dB = dB;
+  b.gu_codes = gu_codes;
+  b.dn_codes = dn_codes;
+  // the nested-form absmax was expanded into the workspace by the training forward
+  b.gu_scales = dq ? static_cast<const void*>(at<float>(ws, L.fwd.gu_absmax)) : gu_scales;
+  b.dn_scales = dq ? static_cast<const void*>(at<float>(ws, L.fwd.dn_absmax)) : dn_scales;
+  b.lora_A = lora_A;
+  b.lora_B = lora_B;
+  return launch_moe_backward(b, reinterpret_cast<cudaStream_t>(stream));
 }
 
 e4b_status e4b_device_status(void* ws, e4b_stream stream) {

@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 
 #include "e4b.h"
+#include "e4b_internal.h"
 
 namespace e4b {
 
@@ -297,18 +298,7 @@ __device__ __forceinline__ uint32_t swizzled_offset(uint32_t row, uint32_t chunk
 }
 
 // ---------------------------------------------------------------------- expert epilogue
-// What the gate_up and down launches add to their fp32 accumulators.  The
-// stock epilogue is silu(gate) * up with no bias.  The gpt-oss epilogue
-// ("How do I train and serve MoE models released in MXFP4 (gpt-oss,
-// DeepSeek-V4)?", "Why it happens": per-expert biases and a clamped GLU) adds
-// a per-expert bias to each output and, on gate_up, applies
-// min(gate, limit) * sigmoid(alpha * .) * (clamp(up, -limit, limit) + beta).
-struct Epilogue {
-  const float* bias;   // gate_up launch: [E, 2I] as [gate | up]; down launch: [E, H]; null = none
-  int32_t glu;         // E4B_ACT_SWIGLU or E4B_ACT_CLAMPED_GLU
-  float alpha, limit, beta;
-};
-
+// (Epilogue, the biases and activation parameters, is declared in e4b_internal.h)
 __device__ __forceinline__ float expert_act(const Epilogue& ep, float gate, float up) {
   if (ep.glu == E4B_ACT_CLAMPED_GLU) {
     const float g = fminf(gate, ep.limit);

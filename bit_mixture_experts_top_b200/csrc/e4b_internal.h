@@ -10,6 +10,19 @@
 
 namespace e4b {
 
+// What the gate_up and down launches add to their fp32 accumulators.  The
+// stock epilogue is silu(gate) * up with no bias.  The gpt-oss epilogue
+// ("How do I train and serve MoE models released in MXFP4 (gpt-oss,
+// DeepSeek-V4)?", "Why it happens": per-expert biases and a clamped GLU) adds
+// a per-expert bias to each output and, on gate_up, applies
+// min(gate, limit) * sigmoid(alpha * .) * (clamp(up, -limit, limit) + beta).
+struct Epilogue {
+  const float* bias;   // gate_up launch: [E, 2I] as [gate | up]; down launch: [E, H]; null = none
+  int32_t glu;         // E4B_ACT_SWIGLU or E4B_ACT_CLAMPED_GLU
+  float alpha, limit, beta;
+};
+
+
 constexpr size_t kAlign = 256;
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 32;
@@ -115,6 +128,7 @@ struct GroupedGemmLaunch {
   const float* bias;        // mode 0: [E, 2I] ([gate | up]); mode 1: [E, H]; null = none
   int32_t glu;              // E4B_ACT_SWIGLU / E4B_ACT_CLAMPED_GLU (mode 0)
   float glu_alpha, glu_limit, glu_beta;
+  float* g_out;             // mode 0: the pre-activation outputs G [R, 2I] fp32 ([gate | up]) or null
 };
 e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 
@@ -124,6 +138,31 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s);
 bool skinny_gemm_supported(int32_t K, int32_t fmt);   // the per-unit scale buffers fit in shared memory
 
 int device_sm_count();
+
+// Layer backward (QLoRA): everything the training forward left in its workspace plus the
+// upstream gradient; outputs dx [T, H], dlogits [T, E] and, with LoRA, dA [E, H, r], dB [E, r, 2I].
+struct BackwardLaunch {
+  int32_t T, k, E, H, I, fmt, gating, lora_rank;
+  float lora_scale;
+  Epilogue ep;
+  const uint16_t* logits;       // [T, E] bf16
+  const uint16_t* dout;         // [T, H] bf16
+  const float* y;               // [R, H] fp32 down outputs (expert order)
+  const float* topk_w;
+  const int32_t *topk_ids, *slot_pos, *sorted_slot, *expert_offsets;
+  const uint16_t* x_sorted;     // [R, H]
+  const uint16_t* xa;           // [R, 64] bf16 s * x A_e (LoRA)
+  const float* G;               // [R, 2I] fp32
+  uint16_t* dY;                 // [R, H] bf16 scratch
+  uint16_t* dG;                 // [R, 2I] bf16 scratch
+  float* dxa;                   // [R, 16] fp32 scratch
+  float* dX;                    // [R, H] fp32 scratch
+  float *dx, *dlogits, *dA, *dB;
+  const uint8_t *gu_codes, *dn_codes;
+  const void *gu_scales, *dn_scales;   // NF4 fp32 absmax (expanded for the nested form) or MXFP4 e8m0
+  const uint16_t *lora_A, *lora_B;
+};
+e4b_status launch_moe_backward(const BackwardLaunch& b, cudaStream_t s);
 
 // 2-D tiled tensor map (inner dim contiguous, `row_bytes` apart) through the
 // driver entry point; false when the driver refuses the description.

@@ -116,6 +116,7 @@ struct Params {
   int32_t* status;
   uint64_t wait_limit_ns;
   Epilogue ep;            // biases and activation
+  float* g_out;           // mode 0: pre-activation outputs G [R, 2I] fp32, or null
   float lut[16];          // NF4 levels
 };
 
@@ -657,6 +658,8 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
             const float u = __shfl_xor_sync(kFull, v, 16);
             if (lane < 16 && c0 + j < t.rows)
               h[static_cast<int64_t>(t.row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(expert_act(p.ep, v, u));
+            if (p.g_out && c0 + j < t.rows)   // kept for the backward: gate (lanes 0-15) or up (16-31)
+              p.g_out[static_cast<int64_t>(t.row0 + c0 + j) * 2 * p.I + (lane < 16 ? 0 : p.I) + f] = v;
           }
         } else {
           const int n = BM * t.nb + 32 * q + lane;
@@ -789,6 +792,7 @@ e4b_status launch_grouped_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.status = g.status;
   prm.wait_limit_ns = g.wait_limit_ns;
   prm.ep = Epilogue{g.bias, g.mode == 0 ? g.glu : E4B_ACT_SWIGLU, g.glu_alpha, g.glu_limit, g.glu_beta};
+  prm.g_out = g.mode == 0 ? g.g_out : nullptr;
   for (int i = 0; i < 16; ++i) prm.lut[i] = nf4_table().level[i];
   switch (BN) {
     case 32: return dispatch_fmt_mode<32>(g, tc, ta, tx, prm, s);

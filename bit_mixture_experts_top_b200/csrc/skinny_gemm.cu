@@ -104,6 +104,7 @@ struct SkParams {
   uint32_t* counters;     // [2]: next unit, CTAs done (zero between launches)
   uint64_t wait_limit_ns;
   Epilogue ep;            // biases and activation
+  float* g_out;           // mode 0: pre-activation outputs G [R, 2I] fp32, or null
   uint32_t level2[8];     // NF4: bf16 levels, two per word (level 2w low half)
 };
 
@@ -575,8 +576,13 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
               if (tok0 + 2 * c + r < un.m) {
-                const float a = expert_act(p.ep, v[r] + b_lo, v[2 + r] + b_hi);
-                h[static_cast<int64_t>(un.t0 + tok0 + 2 * c + r) * p.I + col] = __float2bfloat16_rn(a);
+                const int64_t row = un.t0 + tok0 + 2 * c + r;
+                const float gate = v[r] + b_lo, up = v[2 + r] + b_hi;
+                h[row * p.I + col] = __float2bfloat16_rn(expert_act(p.ep, gate, up));
+                if (p.g_out) {   // kept for the backward
+                  p.g_out[row * 2 * p.I + col] = gate;
+                  p.g_out[row * 2 * p.I + p.I + col] = up;
+                }
               }
             }
           } else {
@@ -666,6 +672,7 @@ e4b_status launch_skinny_gemm(const GroupedGemmLaunch& g, cudaStream_t s) {
   prm.out = g.out;
   prm.status = g.status;
   prm.ep = Epilogue{g.bias, g.mode == 0 ? g.glu : E4B_ACT_SWIGLU, g.glu_alpha, g.glu_limit, g.glu_beta};
+  prm.g_out = g.mode == 0 ? g.g_out : nullptr;
   prm.counters = reinterpret_cast<uint32_t*>(g.status) + 8 + 2 * g.mode;
   prm.wait_limit_ns = g.wait_limit_ns;
   const Nf4Table& t = nf4_table();

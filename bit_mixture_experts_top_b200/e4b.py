@@ -88,6 +88,11 @@ _SIGS = {
                          _sz, _vp], _i32),
     "e4b_moe_forward_stage": ([_i32, ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                _vp, _vp, _vp, _sz, _vp], _i32),
+    "e4b_moe_train_workspace_bytes": ([ctypes.POINTER(MoeDesc), _i32], _sz),
+    "e4b_moe_forward_train": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                               _vp, _sz, _vp], _i32),
+    "e4b_moe_backward": ([ctypes.POINTER(MoeDesc), _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                          _vp, _sz, _vp], _i32),
     "e4b_device_status": ([_vp, _vp], _i32),
     "e4b_debug_wait_timeout": ([_u32, _vp, _sz, _vp], _i32),
 }
@@ -221,6 +226,30 @@ def e4b_moe_forward_stage(stage, desc, T, x, logits, gu_codes, gu_scales, dn_cod
                                        ws.numel() * ws.element_size(), _stream(stream)),
            "e4b_moe_forward_stage")
     return out
+
+
+def e4b_moe_train_workspace_bytes(desc, T):
+    return lib().e4b_moe_train_workspace_bytes(ctypes.byref(desc), T)
+
+
+def e4b_moe_forward_train(desc, T, x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias,
+                          dn_bias, out, ws, stream=None):
+    _need_cuda(x, logits, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, gu_bias, dn_bias, out, ws)
+    _check(lib().e4b_moe_forward_train(ctypes.byref(desc), T, _ptr(x), _ptr(logits), _ptr(gu_codes),
+                                       _ptr(gu_scales), _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A),
+                                       _ptr(lora_B), _ptr(gu_bias), _ptr(dn_bias), _ptr(out), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "e4b_moe_forward_train")
+    return out
+
+
+def e4b_moe_backward(desc, T, logits, dout, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, dx, dlogits,
+                     dA, dB, ws, stream=None):
+    _need_cuda(logits, dout, gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B, dx, dlogits, dA, dB, ws)
+    _check(lib().e4b_moe_backward(ctypes.byref(desc), T, _ptr(logits), _ptr(dout), _ptr(gu_codes), _ptr(gu_scales),
+                                  _ptr(dn_codes), _ptr(dn_scales), _ptr(lora_A), _ptr(lora_B), _ptr(dx),
+                                  _ptr(dlogits), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "e4b_moe_backward")
+    return dx, dlogits, dA, dB
 
 
 def e4b_device_status(ws, stream=None):

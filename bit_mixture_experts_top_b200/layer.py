@@ -70,6 +70,41 @@ class MoeLayer:
                             out, ws, stream)
         return out
 
+    def train_workspace(self, T, device):
+        need = e4b.e4b_moe_train_workspace_bytes(self.desc, T)
+        if need == 0:
+            raise ValueError("e4b: unsupported layer shape")
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=device)
+        return self._ws
+
+    def forward_train(self, x_bits, logits_bits, out=None, stream=None):
+        """The forward, keeping in the workspace what :meth:`backward` needs."""
+        T = x_bits.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x_bits.device)
+        ws = self.train_workspace(T, x_bits.device)
+        e4b.e4b_moe_forward_train(self.desc, T, x_bits, logits_bits, self.gate_up.codes, self.gate_up.scales,
+                                  self.down.codes, self.down.scales, self.lora_A, self.lora_B, self.gu_bias,
+                                  self.dn_bias, out, ws, stream)
+        return out
+
+    def backward(self, logits_bits, dout_bits, stream=None):
+        """Gradients (dx [T, H], dlogits [T, E], dA [E, H, r], dB [E, r, 2I], fp32) of sum(dout * out) for the
+        last :meth:`forward_train`; dA, dB are None without LoRA."""
+        T = logits_bits.shape[0]
+        dev = logits_bits.device
+        dx = torch.empty((T, self.H), dtype=torch.float32, device=dev)
+        dl = torch.empty((T, self.E), dtype=torch.float32, device=dev)
+        dA = dB = None
+        if self.lora_rank:
+            dA = torch.empty((self.E, self.H, self.lora_rank), dtype=torch.float32, device=dev)
+            dB = torch.empty((self.E, self.lora_rank, 2 * self.I), dtype=torch.float32, device=dev)
+        e4b.e4b_moe_backward(self.desc, T, logits_bits, dout_bits, self.gate_up.codes, self.gate_up.scales,
+                             self.down.codes, self.down.scales, self.lora_A, self.lora_B, dx, dl, dA, dB, self._ws,
+                             stream)
+        return dx, dl, dA, dB
+
     def region(self, T, which, dtype):
         off, nbytes = e4b.e4b_moe_workspace_region(self.desc, T, which)
         return self._ws[off:off + nbytes].view(dtype)

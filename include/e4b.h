@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define E4B_ABI_VERSION 2
+#define E4B_ABI_VERSION 3
 
 typedef enum {
   E4B_OK = 0,
@@ -281,6 +281,63 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, int32_t T, const uint16_t* x,
                            const uint16_t* lora_A, const uint16_t* lora_B,
                            const float* gu_bias, const float* dn_bias, uint16_t* out,
                            void* ws, size_t ws_bytes, e4b_stream stream);
+
+/*
+ * QLoRA training: the layer's backward through its frozen 4-bit stacks.
+ * [IX] experts4bit-qlora table: ExpertsLoRA wraps each frozen expert stack
+ * with a per-expert low-rank adapter, and the fast training path runs the
+ * grouped kernels with dgrad, i.e. it also takes the input gradient through
+ * the frozen 4-bit weights.  The packed stacks and any biases are frozen; the
+ * trainable parameters are the LoRA factors, and the layer's inputs (x and
+ * the router logits) receive gradients.  The routing choice is piecewise
+ * constant and carries none; only the gate weights of the chosen experts do.
+ */
+
+/* Workspace bytes of e4b_moe_forward_train + e4b_moe_backward at T tokens (0 on a bad desc). */
+size_t e4b_moe_train_workspace_bytes(const e4b_moe_desc* d, int32_t T);
+
+/*
+ * e4b_moe_forward that also keeps, in its workspace, what e4b_moe_backward
+ * needs: the routing, the routed rows, the down outputs and the gate_up
+ * outputs before the activation (fp32, LoRA delta and bias included).
+ * Arguments as e4b_moe_forward; ws must hold e4b_moe_train_workspace_bytes.
+ */
+e4b_status e4b_moe_forward_train(const e4b_moe_desc* d, int32_t T, const uint16_t* x,
+                                 const uint16_t* logits, const uint8_t* gu_codes, const void* gu_scales,
+                                 const uint8_t* dn_codes, const void* dn_scales,
+                                 const uint16_t* lora_A, const uint16_t* lora_B,
+                                 const float* gu_bias, const float* dn_bias, uint16_t* out,
+                                 void* ws, size_t ws_bytes, e4b_stream stream);
+
+/*
+ * Gradients of sum(dout * out) for the forward last run by
+ * e4b_moe_forward_train on this workspace (same desc, T, stacks, LoRA factors
+ * and logits; nothing in between may reuse the workspace).  For routed row
+ * r = (t, j) of expert e with gate weight w and LoRA scale s = d->lora_scale:
+ *   dY_r = w dout_t;  dh = dY_r W_dn[e];  dG = act'(G) applied to dh;
+ *   dxa = s dG B_e^T;  dx_t = sum_j (dG W_gu[e] + dxa A_e^T);
+ *   dB_e = sum over e's rows of s (x A_e)^T dG;  dA_e = sum of x^T dxa;
+ * and dw_j = <dout_t, y_r> reaches the logits through the gating softmax
+ * (E4B_GATE_SOFTMAX_TOPK: w_j (dw_j - sum_i w_i dw_i) at the picks, 0
+ * elsewhere; E4B_GATE_SOFTMAX_ALL: p_e ([e = id_j] dw_j - sum_i w_i dw_i)).
+ * The clamps of E4B_ACT_CLAMPED_GLU pass the gradient inside their range,
+ * ends included.
+ *   logits  : [T, E] bf16, the forward's                    (device, read)
+ *   dout    : [T, H] bf16 upstream gradient                 (device, read)
+ *   gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B: the forward's
+ *   dx      : [T, H] fp32                                   (device, written)
+ *   dlogits : [T, E] fp32                                   (device, written)
+ *   dA      : [E, H, r] fp32, dB : [E, r, 2I] fp32, with LoRA, else NULL
+ *             (device, written; experts no row is routed to get zeros)
+ *   ws      : the workspace e4b_moe_forward_train filled
+ * Within the forward's tolerance class: bf16 operands (dY, dG and the decoded
+ * weights), fp32 accumulation.
+ */
+e4b_status e4b_moe_backward(const e4b_moe_desc* d, int32_t T, const uint16_t* logits,
+                            const uint16_t* dout, const uint8_t* gu_codes, const void* gu_scales,
+                            const uint8_t* dn_codes, const void* dn_scales,
+                            const uint16_t* lora_A, const uint16_t* lora_B, float* dx, float* dlogits,
+                            float* dA, float* dB, void* ws, size_t ws_bytes, e4b_stream stream);
 
 /* Stages of e4b_moe_forward, in order. */
 enum {

@@ -26,7 +26,7 @@ def test_library_exports_every_declared_function(L):
 
 
 def test_abi_version(L):
-    assert e4b.e4b_abi_version() == 2
+    assert e4b.e4b_abi_version() == 3
     assert L.e4b_status_string(4).decode().startswith("E4B_ERR_TIMEOUT")
 
 
@@ -95,6 +95,31 @@ def test_forward_validation_and_workspace(L):
     off, nb = e4b.e4b_moe_workspace_region(d, 64, e4b.E4B_WS_H)
     assert off % 256 == 0 and nb == 64 * 2 * 128 * 2 and off + nb <= ws
     assert L.e4b_debug_wait_timeout(2_000_000_000, 256, 4096, None) == e4b.E4B_ERR_INVALID_ARG
+
+
+def test_training_entry_validation(L):
+    d = e4b.make_desc(8, 256, 128, 2, "mxfp4", lora_rank=8, lora_scale=2.0)
+    fw = e4b.e4b_moe_workspace_bytes(d, 64)
+    tw = e4b.e4b_moe_train_workspace_bytes(d, 64)
+    # the training workspace adds the saved gate_up outputs (fp32) and the backward's scratch
+    assert tw >= fw + 64 * 2 * (2 * 128 * 4 + 256 * 2 + 2 * 128 * 2 + 16 * 4 + 256 * 4) and tw % 256 == 0
+    assert e4b.e4b_moe_train_workspace_bytes(e4b.make_desc(8, 250, 128, 2, "mxfp4"), 64) == 0
+    fake = 4096
+    # the training forward wants the larger workspace
+    st = L.e4b_moe_forward_train(ctypes.byref(d), 64, fake, fake, fake, fake, fake, fake, fake, fake, None, None,
+                                 fake, fake, fw, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
+    # backward: LoRA factors and their gradients all present or all absent; workspace size; null outputs
+    args = [fake] * 10
+    st = L.e4b_moe_backward(ctypes.byref(d), 64, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            None, fake, fake, tw, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
+    st = L.e4b_moe_backward(ctypes.byref(d), 64, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                            fake, fake, fake, tw - 256, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
+    st = L.e4b_moe_backward(ctypes.byref(d), 64, fake, fake, fake, fake, fake, fake, fake, fake, None, fake,
+                            fake, fake, fake, tw, None)
+    assert st == e4b.E4B_ERR_INVALID_ARG
 
 
 def test_expand_absmax_dq_validation(L):
