@@ -241,12 +241,81 @@ def bench_configs(dev, peaks, max_over_ranks, target_s=0.4):
                 rec[kk]["frac"] = rec[kk]["gbs"] / peaks["hbm_gbs"]
             rec["layer_frac"] = rec["layer_weight_gbs"] / peaks["hbm_gbs"]
             rec["layer_tflops"] = w.flops(T) / (ms * 1e-3) / 1e12
+        if w.lora_rank:
+            rec["training"] = bench_training(lay, layers, w, T, x, lg, wbytes, peaks, max_over_ranks, target_s)
         rows.append(rec)
         del g_fwd, g_gu, g_dn, layers, lay, ws
         torch.cuda.synchronize()
     built.clear()
     torch.cuda.empty_cache()
     return rows
+
+
+def bench_training(lay, layers, w, T, x, lg, wbytes, peaks, max_over_ranks, target_s):
+    """A QLoRA training step on the layer (the forward that keeps what the backward needs, then the backward:
+    LoRA factor gradients and dgrad through both frozen stacks), timed as CUDA-graph replays over the same
+    weight copies as the forward; the backward streams every touched expert's packed weights once more."""
+    import torch
+    from bit_mixture_experts_top_b200 import e4b, synth, layer as lmod
+    dev = x.device
+    ws = lay.train_workspace(T, dev)
+    out = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+    dout = lmod.bits_tensor(synth.normal_bf16((T, w.H), 1.0, w.seed, f"dout{T}"), dev)
+    r = w.lora_rank
+    dx = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+    dl = torch.empty((T, w.E), dtype=torch.float32, device=dev)
+    dA = torch.empty((w.E, w.H, r), dtype=torch.float32, device=dev)
+    dB = torch.empty((w.E, r, 2 * w.I), dtype=torch.float32, device=dev)
+
+    def fwd(l):
+        e4b.e4b_moe_forward_train(l.desc, T, x, lg, l.gate_up.codes, l.gate_up.scales, l.down.codes, l.down.scales,
+                                  l.lora_A, l.lora_B, None, None, out, ws)
+
+    def bwd(l):
+        e4b.e4b_moe_backward(l.desc, T, lg, dout, l.gate_up.codes, l.gate_up.scales, l.down.codes, l.down.scales,
+                             l.lora_A, l.lora_B, dx, dl, dA, dB, ws)
+
+    def graph_of(fn):
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    g_step = graph_of(lambda: [(fwd(l), bwd(l)) for l in layers])
+    g_bwd = graph_of(lambda: [bwd(l) for l in layers])
+
+    def per_layer_ms(g):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        n = int(min(500, max(5, target_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+        e0.record()
+        for _ in range(n):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1) / (n * len(layers)))
+
+    step_ms = per_layer_ms(g_step)
+    bwd_ms = per_layer_ms(g_bwd)
+    if e4b.e4b_device_status(ws) != e4b.E4B_OK:
+        raise RuntimeError("device status reported an error in the training step")
+    del g_step, g_bwd
+    gbs = wbytes / (bwd_ms * 1e-3) / 1e9
+    return {"step_ms": step_ms, "tokens_per_s": T / (step_ms * 1e-3), "backward_ms": bwd_ms,
+            "backward_weight_gbs": gbs, "backward_frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "note": "forward keeping G + backward (dx, dlogits, dA, dB); weight bytes = touched experts' packed "
+                    "stacks, streamed once by the backward's two dgrad launches"}
 
 
 def init_dist():

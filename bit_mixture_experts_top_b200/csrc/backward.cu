@@ -36,9 +36,11 @@ namespace {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr int kDgTok = 64;       // routed rows per dgrad tile
-constexpr int kDgCols = 64;      // output columns per dgrad tile
+constexpr int kDgCols = 128;     // output columns per dgrad tile
 constexpr int kDgK = 64;         // stored rows (contraction) per slab
-constexpr int kPad = 72;         // shared tile row pitch in bf16 (conflict-free matrix loads)
+constexpr int kPad = 72;         // activation tile row pitch in bf16 (conflict-free matrix loads)
+constexpr int kPadW = 136;       // weight tile row pitch in bf16
+constexpr int kDgSmem = 2 * kDgK * kPadW * 2 + 2 * kDgTok * kPad * 2;   // double-buffered tiles
 
 __device__ __forceinline__ float sigmoidf_acc(float z) { return 1.0f / (1.0f + expf(-z)); }
 
@@ -238,13 +240,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// out[r, n] = sum_m act[r, m] * W[e][m, n] for one (64 routed rows) x (64 columns)
-// tile, then the mode's epilogue.  256 threads: warp (wt, wn) owns rows
-// 16wt..16wt+15 and columns 32wn..32wn+31 of the tile.
+// out[r, n] = sum_m act[r, m] * W[e][m, n] for one (64 routed rows) x (128
+// columns) tile, then the mode's epilogue.  256 threads: warp (wt, wn) owns
+// rows 16wt..16wt+15 and columns 64wn..64wn+63.  The stored rows go by in
+// slabs of 64; the next slab's codes, scales and activation rows are loaded
+// into registers while the current one is multiplied, and the decoded tiles
+// are double-buffered in shared memory (one barrier per slab).
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
-  __shared__ __align__(16) uint16_t sW[kDgK][kPad];      // decoded slab [stored row m][column n]
-  __shared__ __align__(16) uint16_t sA[kDgTok][kPad];    // activation slab [routed row][stored row m]
+  extern __shared__ __align__(16) uint8_t dg_smem[];
+  uint16_t (*sW)[kDgK][kPadW] = reinterpret_cast<uint16_t (*)[kDgK][kPadW]>(dg_smem);                 // [2][m][n]
+  uint16_t (*sA)[kDgTok][kPad] = reinterpret_cast<uint16_t (*)[kDgTok][kPad]>(dg_smem + 2 * kDgK * kPadW * 2);
   __shared__ float s_lut[16];
   __shared__ int s_tile[3];
   if (FMT == E4B_NF4 && threadIdx.x < 16) s_lut[threadIdx.x] = p.lut[threadIdx.x];
@@ -256,61 +262,75 @@ __global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wt = warp & 3, wn = warp >> 2;
   const int g = lane >> 2, c = lane & 3;
-  // loader roles: stored row lm = tid / 4, 16 columns (8 code bytes) at 16 * ls
+  // loader: stored row lm = tid / 4, 32 columns (16 code bytes) at 32 * ls; those columns
+  // lie in one quantisation block and are either all inside the stack or all past its end
   const int lm = tid >> 2, ls = tid & 3;
+  const bool col_ok = n0 + 32 * ls < p.N;
   const int64_t row_bytes = p.N / 2;
-  const uint8_t* cbase = p.codes + (static_cast<int64_t>(e) * p.M + lm) * row_bytes + n0 / 2 + 8 * ls;
-  // activation loader: routed row lr = tid / 4 (clamped into the tile), 16 stored rows at 16 * ls
+  const uint8_t* cbase = p.codes + (static_cast<int64_t>(e) * p.M + lm) * row_bytes + n0 / 2 + 16 * ls;
+  const int64_t ebase = (static_cast<int64_t>(e) * p.M + lm) * p.N + n0 + 32 * ls;    // element index at m0 = 0
+  // activation rows: routed row lr = tid / 4 (clamped into the tile), 16 stored rows at 16 * ls
   const int lr = min(tid >> 2, rows - 1);
   const uint16_t* abase = p.act + static_cast<int64_t>(r0 + lr) * p.M + 16 * ls;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
-
-  for (int m0 = 0; m0 < p.M; m0 += kDgK) {
-    // decode one 64 x 64 slab of W[e] into bf16
-    const uint2 q = __ldg(reinterpret_cast<const uint2*>(cbase + static_cast<int64_t>(m0) * row_bytes));
-    const int64_t elem0 = (static_cast<int64_t>(e) * p.M + m0 + lm) * p.N + n0 + 16 * ls;   // first element
-    uint32_t w[8];
-    if (FMT == E4B_NF4) {
-      const float a = __ldg(static_cast<const float*>(p.scales) + elem0 / 64);
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const uint32_t by = ((b < 4 ? q.x : q.y) >> (8 * (b & 3))) & 0xFFu;   // element 2b high, 2b+1 low
-        w[b] = pack_bf16x2(s_lut[by >> 4] * a, s_lut[by & 15u] * a);
-      }
-    } else {
-      const float sc = e8m0_f32(__ldg(static_cast<const uint8_t*>(p.scales) + elem0 / 32));
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        const uint32_t by = ((b < 4 ? q.x : q.y) >> (8 * (b & 3))) & 0xFFu;   // element 2b low, 2b+1 high
-        w[b] = pack_bf16x2(e2m1_f32(by & 15u) * sc, e2m1_f32(by >> 4) * sc);
-      }
+  uint4 qn = make_uint4(0u, 0u, 0u, 0u), an0, an1;
+  float sn = 0.0f;
+  auto load = [&](int m0) {
+    if (col_ok) {
+      qn = __ldg(reinterpret_cast<const uint4*>(cbase + static_cast<int64_t>(m0) * row_bytes));
+      const int64_t el = ebase + static_cast<int64_t>(m0) * p.N;
+      sn = FMT == E4B_NF4 ? __ldg(static_cast<const float*>(p.scales) + el / 64)
+                          : e8m0_f32(__ldg(static_cast<const uint8_t*>(p.scales) + el / 32));
     }
-    const uint4 a0 = __ldg(reinterpret_cast<const uint4*>(abase + m0));
-    const uint4 a1 = __ldg(reinterpret_cast<const uint4*>(abase + m0) + 1);
-    __syncthreads();                                     // the previous slab is consumed
-    *reinterpret_cast<uint4*>(&sW[lm][16 * ls]) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint4*>(&sW[lm][16 * ls + 8]) = make_uint4(w[4], w[5], w[6], w[7]);
-    *reinterpret_cast<uint4*>(&sA[tid >> 2][16 * ls]) = a0;
-    *reinterpret_cast<uint4*>(&sA[tid >> 2][16 * ls + 8]) = a1;
-    __syncthreads();
+    an0 = __ldg(reinterpret_cast<const uint4*>(abase + m0));
+    an1 = __ldg(reinterpret_cast<const uint4*>(abase + m0) + 1);
+  };
+  auto store = [&](int buf) {          // decode the registers' slab into buffer buf
+    const uint32_t wd[4] = {qn.x, qn.y, qn.z, qn.w};
+    uint32_t w[16];
+#pragma unroll
+    for (int b = 0; b < 16; ++b) {
+      const uint32_t by = (wd[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+      if (FMT == E4B_NF4)        // element 2b in the high nibble; one rounding of level * absmax
+        w[b] = pack_bf16x2(s_lut[by >> 4] * sn, s_lut[by & 15u] * sn);
+      else                       // element 2b in the low nibble; exact
+        w[b] = pack_bf16x2(e2m1_f32(by & 15u) * sn, e2m1_f32(by >> 4) * sn);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint4*>(&sW[buf][lm][32 * ls + 8 * i]) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2],
+                                                                             w[4 * i + 3]);
+    *reinterpret_cast<uint4*>(&sA[buf][tid >> 2][16 * ls]) = an0;
+    *reinterpret_cast<uint4*>(&sA[buf][tid >> 2][16 * ls + 8]) = an1;
+  };
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+  const int nslab = p.M / kDgK;
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int s = 0; s < nslab; ++s) {
+    const int buf = s & 1;
+    if (s + 1 < nslab) load((s + 1) * kDgK);
 #pragma unroll
     for (int kk = 0; kk < kDgK / 16; ++kk) {
-      uint32_t af[4], b01[4], b23[4];
-      ldsm_x4(af, &sA[16 * wt + (lane & 15)][16 * kk + 8 * (lane >> 4)]);
-      ldsm_x4_t(b01, &sW[16 * kk + (lane & 15)][32 * wn + 8 * (lane >> 4)]);
-      ldsm_x4_t(b23, &sW[16 * kk + (lane & 15)][32 * wn + 16 + 8 * (lane >> 4)]);
-      mma16816(acc[0], af, b01[0], b01[1]);
-      mma16816(acc[1], af, b01[2], b01[3]);
-      mma16816(acc[2], af, b23[0], b23[1]);
-      mma16816(acc[3], af, b23[2], b23[3]);
+      uint32_t af[4];
+      ldsm_x4(af, &sA[buf][16 * wt + (lane & 15)][16 * kk + 8 * (lane >> 4)]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t b[4];
+        ldsm_x4_t(b, &sW[buf][16 * kk + (lane & 15)][64 * wn + 16 * q + 8 * (lane >> 4)]);
+        mma16816(acc[2 * q], af, b[0], b[1]);
+        mma16816(acc[2 * q + 1], af, b[2], b[3]);
+      }
     }
+    if (s + 1 < nslab) store(buf ^ 1);
+    __syncthreads();
   }
 
-  // epilogue: acc[nt][h * 2 + i] is row 16wt + g + 8h, column 32wn + 8nt + 2c + i of the tile
+  // epilogue: acc[nt][h * 2 + i] is row 16wt + g + 8h, column 64wn + 8nt + 2c + i of the tile
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
+  for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int tr = 16 * wt + g + 8 * h;
@@ -318,7 +338,8 @@ __global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
       const int64_t r = r0 + tr;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const int n = n0 + 32 * wn + 8 * nt + 2 * c + i;
+        const int n = n0 + 64 * wn + 8 * nt + 2 * c + i;
+        if (n >= p.N) continue;
         const float v = acc[nt][2 * h + i];
         if (MODE == 0) {
           const int64_t gi = r * 2 * p.I + n;
@@ -439,11 +460,19 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float* __restrict
   reinterpret_cast<float4*>(dx + t * H)[c] = acc;
 }
 
+template <int FMT, int MODE>
+cudaError_t launch_dgrad_typed(const DgParams& prm, dim3 grid, cudaStream_t s) {
+  static cudaError_t attr = cudaFuncSetAttribute(dgrad_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kDgSmem);
+  if (attr != cudaSuccess) return attr;
+  return launch_pdl(dgrad_kernel<FMT, MODE>, grid, dim3(256), kDgSmem, s, prm);
+}
+
 template <int MODE>
 cudaError_t launch_dgrad_mode(int32_t fmt, const DgParams& prm, int R, cudaStream_t s) {
-  const dim3 grid(prm.N / kDgCols, (R + kDgTok - 1) / kDgTok + prm.E);
-  if (fmt == E4B_NF4) return launch_pdl(dgrad_kernel<E4B_NF4, MODE>, grid, dim3(256), 0, s, prm);
-  return launch_pdl(dgrad_kernel<E4B_MXFP4, MODE>, grid, dim3(256), 0, s, prm);
+  const dim3 grid((prm.N + kDgCols - 1) / kDgCols, (R + kDgTok - 1) / kDgTok + prm.E);
+  return fmt == E4B_NF4 ? launch_dgrad_typed<E4B_NF4, MODE>(prm, grid, s)
+                        : launch_dgrad_typed<E4B_MXFP4, MODE>(prm, grid, s);
 }
 
 }  // namespace
