@@ -87,9 +87,15 @@ __device__ __forceinline__ float block_max(float v, float* s_red) {
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ float bf16_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
-// One block per token: dw_j = <dout_t, y_(t,j)>, dY rows in expert order, and the
-// logit gradient through the gating softmax (fp32 throughout).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// One block per token: dw_j = <dout_t, y_(t,j)> (one warp per pick j), dY rows
+// in expert order, and the logit gradient through the gating softmax (fp32).
 __global__ void __launch_bounds__(256) bwd_gate_kernel(const uint16_t* __restrict__ dout, const float* __restrict__ y,
                                                        const float* __restrict__ topk_w,
                                                        const int32_t* __restrict__ topk_ids,
@@ -102,20 +108,26 @@ __global__ void __launch_bounds__(256) bwd_gate_kernel(const uint16_t* __restric
   __shared__ float s_red[8];
   __shared__ float s_dw[kMaxTopK];
   const int64_t t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint16_t* drow = dout + t * H;
-  for (int j = 0; j < k; ++j) {
+  for (int j = warp; j < k; j += 8) {
     const int64_t pos = slot_pos[t * k + j];
     const float w = topk_w[t * k + j];
-    const float* yr = y + pos * H;
-    uint16_t* dyr = dY + pos * H;
+    const float4* yr = reinterpret_cast<const float4*>(y + pos * H);
+    const uint2* dr = reinterpret_cast<const uint2*>(drow);
+    uint2* dyr = reinterpret_cast<uint2*>(dY + pos * H);
     float acc = 0.0f;
-    for (int c = threadIdx.x; c < H; c += blockDim.x) {
-      const float d = bf16_to_f32(drow[c]);
-      acc = fmaf(d, yr[c], acc);
-      dyr[c] = __bfloat16_as_ushort(__float2bfloat16_rn(w * d));
+    for (int c = lane; c < H / 4; c += 32) {          // four elements per lane and step
+      const uint2 d = __ldg(dr + c);
+      const float4 v = yr[c];
+      const float d0 = bf16_to_f32(d.x & 0xFFFFu), d1 = bf16_to_f32(d.x >> 16);
+      const float d2 = bf16_to_f32(d.y & 0xFFFFu), d3 = bf16_to_f32(d.y >> 16);
+      acc = fmaf(d0, v.x, fmaf(d1, v.y, fmaf(d2, v.z, fmaf(d3, v.w, acc))));
+      dyr[c] = make_uint2(pack_bf16x2(w * d0, w * d1), pack_bf16x2(w * d2, w * d3));
     }
-    const float dw = block_sum(acc, s_red);
-    if (threadIdx.x == 0) s_dw[j] = dw;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(kFull, acc, off);
+    if (lane == 0) s_dw[j] = acc;
   }
   __syncthreads();
   float S = 0.0f;                                   // sum_j w_j dw_j
@@ -235,10 +247,6 @@ __device__ __forceinline__ float e8m0_f32(uint32_t s) {
   return __uint_as_float(s == 0u ? 0x00400000u : (s == 255u ? 0x7FC00000u : (s << 23)));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
 
 // out[r, n] = sum_m act[r, m] * W[e][m, n] for one (64 routed rows) x (128
 // columns) tile, then the mode's epilogue.  256 threads: warp (wt, wn) owns
@@ -361,27 +369,48 @@ __global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
   }
 }
 
-// dxa[r, j] = s * sum_n dG[r, n] B_e[j, n], one warp per routed row (j < rank; fp32 [R, 16]).
+// dxa[r, j] = s * sum_n dG[r, n] B_e[j, n], one warp per routed row (j < rank;
+// fp32 [R, 16]).  The block's 8 rows are consecutive in expert order: B_e of its
+// first row is staged in shared memory (rows of another expert read global memory).
 __global__ void __launch_bounds__(256) lora_dxa_kernel(const uint16_t* __restrict__ dG, const uint16_t* __restrict__ B,
                                                        const int32_t* __restrict__ sorted_slot,
                                                        const int32_t* __restrict__ topk_ids, int R, int I2, int rank,
-                                                       float scale, float* __restrict__ dxa) {
+                                                       float scale, float* __restrict__ dxa, int stage_b) {
   pdl_wait();
   pdl_launch_dependents();
+  extern __shared__ __align__(16) uint16_t s_B[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 8;
+  int e_cached = -1;
+  if (stage_b) {
+    e_cached = topk_ids[sorted_slot[r0 < R ? r0 : R - 1]];
+    const uint4* gb = reinterpret_cast<const uint4*>(B + static_cast<int64_t>(e_cached) * rank * I2);
+    uint4* sb = reinterpret_cast<uint4*>(s_B);
+    for (int i = threadIdx.x; i < rank * I2 / 8; i += blockDim.x) sb[i] = __ldg(gb + i);
+    __syncthreads();
+  }
+  const int64_t r = r0 + warp;
   if (r >= R) return;
   const int e = topk_ids[sorted_slot[r]];
-  const uint16_t* gr = dG + r * I2;
-  const uint16_t* Be = B + static_cast<int64_t>(e) * rank * I2;
+  const uint16_t* Be = e == e_cached ? s_B : B + static_cast<int64_t>(e) * rank * I2;
+  const uint4* gr = reinterpret_cast<const uint4*>(dG + r * I2);
   float acc[kMaxLoraRank];
 #pragma unroll
   for (int j = 0; j < kMaxLoraRank; ++j) acc[j] = 0.0f;
-  for (int n = lane; n < I2; n += 32) {
-    const float d = bf16_to_f32(gr[n]);
+  for (int v = lane; v < I2 / 8; v += 32) {           // eight columns per lane and step
+    const uint4 d = __ldg(gr + v);
+    const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
-    for (int j = 0; j < kMaxLoraRank; ++j)
-      if (j < rank) acc[j] = fmaf(d, bf16_to_f32(Be[static_cast<int64_t>(j) * I2 + n]), acc[j]);
+    for (int j = 0; j < kMaxLoraRank; ++j) {
+      if (j < rank) {
+        const uint4 b = *reinterpret_cast<const uint4*>(Be + static_cast<int64_t>(j) * I2 + 8 * v);
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          acc[j] = fmaf(bf16_to_f32(dw[q] & 0xFFFFu), bf16_to_f32(bw[q] & 0xFFFFu),
+                        fmaf(bf16_to_f32(dw[q] >> 16), bf16_to_f32(bw[q] >> 16), acc[j]));
+      }
+    }
   }
 #pragma unroll
   for (int j = 0; j < kMaxLoraRank; ++j) {
@@ -508,8 +537,17 @@ e4b_status launch_moe_backward(const BackwardLaunch& b, cudaStream_t s) {
   p.dG = b.dG;
   if (launch_dgrad_mode<0>(b.fmt, p, R, s) != cudaSuccess) return E4B_ERR_CUDA;
   if (b.lora_rank > 0) {
-    if (launch_pdl(lora_dxa_kernel, dim3((R + 7) / 8), dim3(256), 0, s, static_cast<const uint16_t*>(b.dG), b.lora_B,
-                   b.sorted_slot, b.topk_ids, R, I2, b.lora_rank, b.lora_scale, b.dxa) != cudaSuccess)
+    constexpr size_t kStageMax = 200 * 1024;          // B_e in shared memory up to this size
+    size_t smem = static_cast<size_t>(b.lora_rank) * I2 * 2;
+    if (smem > kStageMax) smem = 0;
+    if (smem > 48 * 1024) {
+      static cudaError_t attr = cudaFuncSetAttribute(lora_dxa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     static_cast<int>(kStageMax));
+      if (attr != cudaSuccess) return E4B_ERR_CUDA;
+    }
+    if (launch_pdl(lora_dxa_kernel, dim3((R + 7) / 8), dim3(256), smem, s, static_cast<const uint16_t*>(b.dG),
+                   b.lora_B, b.sorted_slot, b.topk_ids, R, I2, b.lora_rank, b.lora_scale, b.dxa,
+                   smem > 0 ? 1 : 0) != cudaSuccess)
       return E4B_ERR_CUDA;
   }
   // dX = dG W_gu[e] (+ dxa A_e^T) over the gate_up stack's 2I stored rows
