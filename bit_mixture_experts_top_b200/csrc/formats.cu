@@ -12,6 +12,9 @@
 // 2^(s-127) (s = 0 is the fp32 subnormal 2^-127, s = 255 NaN).  The product is
 // exact in fp32 and in bf16 unless it overflows, so one round-to-nearest
 // conversion reproduces the definition bit for bit.
+#include <cmath>
+#include <cstring>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -66,14 +69,25 @@ __global__ void __launch_bounds__(256) dequant_mxfp4_kernel(const uint32_t* __re
   }
 }
 
-struct Nf4Mids {
-  float m[15];
+// Exact decision table for the NF4 code of a quotient y in [-1, 1]: the code
+// is #{i : y > m_i} over the 15 midpoints.  |y| in [2^-5, 1] falls in one of 161
+// buckets given by its exponent and the top five mantissa bits (exact float
+// boundaries [lo, hi)); each bucket holds at most one midpoint (buckets are at
+// most 1/64 wide, midpoints at least 0.08 apart), so per bucket and sign
+// code = base + (y > mid): positive y counts the midpoints below lo and tests
+// the one in [lo, hi); negative y counts those at or below -hi and tests the
+// one in (-hi, -lo].  |y| < 2^-5 lies between the two midpoints next to zero:
+// code 7.  The host builds and checks the table (nf4_bucket_table).
+constexpr int kNf4Buckets = 161;
+constexpr uint32_t kNf4BucketBias = 122u << 5;        // exponent of 2^-5, five mantissa bits
+struct Nf4Buckets {
+  uint2 e[2][kNf4Buckets];                            // [sign][bucket]: {midpoint bits (or +inf), base}
 };
 
 // One half-warp per 64-block: each lane holds 4 consecutive fp32 (16 bytes),
 // the half-warp reduces |x| to absmax, each lane emits 4 codes (2 bytes).
-__device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_t half_mask, float m7,
-                                              const float* s_mid, uint16_t* __restrict__ codes,
+__device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_t half_mask,
+                                              const uint2 (*s_tab)[kNf4Buckets], uint16_t* __restrict__ codes,
                                               float* __restrict__ absmax) {
   float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
@@ -94,11 +108,14 @@ __device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_
     } else {
       const float q = xv[i] * r;
       const float y = fmaf(fmaf(-a, q, xv[i]), r, q);
-      uint32_t k = (y > m7) ? 8u : 0u;        // count of midpoints below y, by bisection
-      k += (y > s_mid[k + 3]) ? 4u : 0u;
-      k += (y > s_mid[k + 1]) ? 2u : 0u;
-      k += (y > s_mid[k]) ? 1u : 0u;
-      c[i] = k;
+      const uint32_t bits = __float_as_uint(y);
+      const int j = static_cast<int>(((bits & 0x7FFFFFFFu) >> 18) - kNf4BucketBias);
+      if (j < 0) {
+        c[i] = 7u;
+      } else {
+        const uint2 t = s_tab[bits >> 31][j];
+        c[i] = t.y + (y > __uint_as_float(t.x) ? 1u : 0u);
+      }
     }
   }
   const uint32_t b0 = (c[0] << 4) | c[1];
@@ -110,11 +127,10 @@ __device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_
 // Each thread takes two quads per trip (q and q + stride): two loads in flight.
 __global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restrict__ x, int64_t quads,
                                                              uint16_t* __restrict__ codes,
-                                                             float* __restrict__ absmax, Nf4Mids mids) {
-  __shared__ float s_mid[16];
-  if (threadIdx.x < 15) s_mid[threadIdx.x] = mids.m[threadIdx.x];
+                                                             float* __restrict__ absmax, const Nf4Buckets tab) {
+  __shared__ uint2 s_tab[2][kNf4Buckets];
+  for (int i = threadIdx.x; i < 2 * kNf4Buckets; i += blockDim.x) (&s_tab[0][0])[i] = (&tab.e[0][0])[i];
   __syncthreads();
-  const float m7 = mids.m[7];
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16u);   // this half-warp only
   // quads and the stride are multiples of 16, so every half-warp stays inside one
@@ -123,8 +139,8 @@ __global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restr
     const int64_t q2 = q + stride;
     const float4 v = __ldcs(x + q);
     const float4 v2 = q2 < quads ? __ldcs(x + q2) : make_float4(0.f, 0.f, 0.f, 0.f);
-    quantize_quad(v, q, half_mask, m7, s_mid, codes, absmax);
-    if (q2 < quads) quantize_quad(v2, q2, half_mask, m7, s_mid, codes, absmax);
+    quantize_quad(v, q, half_mask, s_tab, codes, absmax);
+    if (q2 < quads) quantize_quad(v2, q2, half_mask, s_tab, codes, absmax);
   }
 }
 
@@ -243,13 +259,47 @@ cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, in
   return cudaGetLastError();
 }
 
+namespace {
+
+// The bucket table of quantize_quad, from the fp32 midpoints; null if a premise fails
+// (a bucket with two midpoints, or a midpoint within 2^-5 of zero).
+const Nf4Buckets* nf4_bucket_table() {
+  static Nf4Buckets tab;
+  static bool ok = [] {
+    const float* m = nf4_table().mid;
+    if (!(m[6] < -0x1p-5f && m[7] > 0x1p-5f)) return false;
+    for (int j = 0; j < kNf4Buckets; ++j) {
+      const float lo = std::ldexp(1.0f + static_cast<float>(j % 32) / 32.0f, j / 32 - 5);
+      const float hi = lo + std::ldexp(1.0f / 32.0f, j / 32 - 5);
+      uint32_t base_p = 0, base_n = 0, inpos = 0, inneg = 0;
+      float mid_p = INFINITY, mid_n = INFINITY;
+      for (int i = 0; i < 15; ++i) {
+        if (m[i] < lo) ++base_p;
+        if (m[i] >= lo && m[i] < hi) { mid_p = m[i]; ++inpos; }
+        if (m[i] <= -hi) ++base_n;
+        if (m[i] > -hi && m[i] <= -lo) { mid_n = m[i]; ++inneg; }
+      }
+      if (inpos > 1 || inneg > 1) return false;
+      uint32_t bp, bn;
+      std::memcpy(&bp, &mid_p, 4);
+      std::memcpy(&bn, &mid_n, 4);
+      tab.e[0][j] = make_uint2(bp, base_p);
+      tab.e[1][j] = make_uint2(bn, base_n);
+    }
+    return true;
+  }();
+  return ok ? &tab : nullptr;
+}
+
+}  // namespace
+
 cudaError_t launch_quantize_nf4(const float* x, int64_t n, uint8_t* codes, float* absmax, cudaStream_t s) {
   const int64_t quads = n / 4;
   if (quads == 0) return cudaSuccess;
-  Nf4Mids m;
-  for (int i = 0; i < 15; ++i) m.m[i] = nf4_table().mid[i];
+  const Nf4Buckets* tab = nf4_bucket_table();
+  if (!tab) return cudaErrorInvalidValue;
   quantize_nf4_kernel<<<grid_for(quads, 256, 8), 256, 0, s>>>(reinterpret_cast<const float4*>(x), quads,
-                                                              reinterpret_cast<uint16_t*>(codes), absmax, m);
+                                                              reinterpret_cast<uint16_t*>(codes), absmax, *tab);
   return cudaGetLastError();
 }
 
