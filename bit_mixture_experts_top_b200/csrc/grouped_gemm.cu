@@ -32,7 +32,8 @@
 //   warps 3-10  dequant: 4-bit codes + per-block scale -> bf16 rows written
 //               into tensor memory (tcgen05.st) or 128-byte-swizzled shared
 //               memory, the UMMA A operand;
-//   warps 11-14 epilogue: tcgen05.ld, SwiGLU or fp32 store.
+//   warps 11-14 epilogue: tcgen05.ld, activation and bf16 store (gate_up) or
+//               bias and fp32 store (down).
 // Every wait is bounded: on timeout the kernel records E4B_ERR_TIMEOUT, lets
 // copies and MMAs in flight land, frees its TMEM and returns.
 #include <cuda.h>
@@ -146,15 +147,18 @@ __device__ __forceinline__ bool get_tile(const Params& p, const int32_t* s_chunk
   return true;
 }
 
-// Row of the weight stack behind A-tile row `prow` (mode 0 pairs gate and up
-// rows: within each 32-row group, rows 0..15 are gate features and 16..31 the
-// matching up features) and its row in the raw code tile.
+// Row of the weight stack behind A-tile row `prow` and its row in the raw code
+// tile.  Mode 0 pairs gate and up rows: within each 32-row group (one epilogue
+// warp's TMEM lanes), rows 0..15 are gate features and 16..31 the matching up
+// features, and within each half row r < 8 is feature 2r and row r + 8 feature
+// 2r + 1, so a 16x256b TMEM load hands every thread two adjacent features.
 template <int MODE>
 __device__ __forceinline__ void tile_row(const Params& p, int nb, int prow, int& wrow, int& raw_row) {
   if (MODE == 0) {
     const int g = prow >> 5, wi = prow & 31;
-    const int f = 64 * nb + 16 * g + (wi & 15);
-    raw_row = (wi < 16 ? 0 : 64) + 16 * g + (wi & 15);
+    const int fi = 2 * (wi & 7) + ((wi >> 3) & 1);
+    const int f = 64 * nb + 16 * g + fi;
+    raw_row = (wi < 16 ? 0 : 64) + 16 * g + fi;
     wrow = (wi < 16) ? f : p.I + f;
   } else {
     raw_row = prow;
@@ -642,30 +646,60 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1)
       if (!mbar_wait_sleep(&acc_full[buf], aphase, wctx, 401, 256)) break;
       tc_fence_after_sync();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * BN);
-      for (int c0 = 0; c0 < BN && c0 < t.rows; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr + c0, r);
-        tmem_ld_wait();
-        if (MODE == 0) {
-          const int f = 64 * t.nb + 16 * q + (lane & 15);
-          __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
-          // lanes 0-15 hold gate rows, lanes 16-31 the matching up rows
-          const float bv = p.ep.bias ? __ldg(p.ep.bias + static_cast<int64_t>(t.e) * 2 * p.I + (lane < 16 ? 0 : p.I) + f)
-                                     : 0.f;
+      if constexpr (MODE == 0) {
+        // Thread t holds the adjacent features f, f + 1 (rows t/4 and t/4 + 8 of
+        // the gate slab, lanes 32q..32q+15, and of the up slab, 32q+16..32q+31)
+        // for the tokens 8i + 2(t%4) + {0, 1} of each 32-column chunk: the
+        // activation of every (feature, token) is formed in the thread that holds
+        // its gate and up values, and two features go out in one 4-byte store.
+        const int f = 64 * t.nb + 16 * q + 2 * (lane >> 2);
+        const int tc = 2 * (lane & 3);
+        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out);
+        float bg0 = 0.f, bg1 = 0.f, bu0 = 0.f, bu1 = 0.f;
+        if (p.ep.bias) {
+          const float* b = p.ep.bias + static_cast<int64_t>(t.e) * 2 * p.I + f;
+          bg0 = __ldg(b);
+          bg1 = __ldg(b + 1);
+          bu0 = __ldg(b + p.I);
+          bu1 = __ldg(b + p.I + 1);
+        }
+        for (int c0 = 0; c0 < BN && c0 < t.rows; c0 += 32) {
+          uint32_t g[16], u[16];
+          tmem_ld_16x256b_x4(taddr + c0, g);
+          tmem_ld_16x256b_x4(taddr + (16u << 16) + c0, u);
+          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float v = __uint_as_float(r[j]) + bv;
-            const float u = __shfl_xor_sync(kFull, v, 16);
-            if (lane < 16 && c0 + j < t.rows)
-              h[static_cast<int64_t>(t.row0 + c0 + j) * p.I + f] = __float2bfloat16_rn(expert_act(p.ep, v, u));
-            if (p.g_out && c0 + j < t.rows)   // kept for the backward: gate (lanes 0-15) or up (16-31)
-              p.g_out[static_cast<int64_t>(t.row0 + c0 + j) * 2 * p.I + (lane < 16 ? 0 : p.I) + f] = v;
+          for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int tok = c0 + 8 * i + tc + hh;
+              if (tok < t.rows) {
+                const float g0 = __uint_as_float(g[4 * i + hh]) + bg0;
+                const float g1 = __uint_as_float(g[4 * i + 2 + hh]) + bg1;
+                const float u0 = __uint_as_float(u[4 * i + hh]) + bu0;
+                const float u1 = __uint_as_float(u[4 * i + 2 + hh]) + bu1;
+                const int64_t row = t.row0 + tok;
+                *reinterpret_cast<__nv_bfloat162*>(h + row * p.I + f) =
+                    __floats2bfloat162_rn(expert_act(p.ep, g0, u0), expert_act(p.ep, g1, u1));
+                if (p.g_out) {              // kept for the backward: pre-activation gate and up
+                  float* go = p.g_out + row * 2 * p.I + f;
+                  *reinterpret_cast<float2*>(go) = make_float2(g0, g1);
+                  *reinterpret_cast<float2*>(go + p.I) = make_float2(u0, u1);
+                }
+              }
+            }
           }
-        } else {
-          const int n = BM * t.nb + 32 * q + lane;
-          float* y = reinterpret_cast<float*>(p.out);
+        }
+      } else {
+        // lane = output feature n, one 128-byte row segment per store
+        const int n = BM * t.nb + 32 * q + lane;
+        float* y = reinterpret_cast<float*>(p.out);
+        const float bv = (p.ep.bias && n < p.N) ? __ldg(p.ep.bias + static_cast<int64_t>(t.e) * p.N + n) : 0.f;
+        for (int c0 = 0; c0 < BN && c0 < t.rows; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(taddr + c0, r);
+          tmem_ld_wait();
           if (n < p.N) {
-            const float bv = p.ep.bias ? __ldg(p.ep.bias + static_cast<int64_t>(t.e) * p.N + n) : 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j)
               if (c0 + j < t.rows) y[static_cast<int64_t>(t.row0 + c0 + j) * p.N + n] = __uint_as_float(r[j]) + bv;

@@ -142,3 +142,49 @@ def test_quantize_nf4_qwen3_stack_sampled():
     rc, ra = onf4.quantize_nf4(w.reshape(-1, 64)[blocks].reshape(-1))
     assert np.array_equal(ga.view(np.uint32), ra.view(np.uint32))
     assert np.array_equal(gc.reshape(-1), rc)
+
+
+def test_quantize_nf4_every_absmax_significand_near_midpoints():
+    """Every fp32 significand of the absmax (a in [1, 2): scaling by a power of two changes no quotient),
+    with elements a * m (rounded) moved -3..+3 ulp for each of the 15 decision midpoints m and both signs:
+    210 quotients within a few ulps of a decision per significand, 2^23 significands.  The expected code
+    is the count of midpoints strictly below the IEEE fp32 quotient, computed with torch's correctly
+    rounded device division and a left-sided bucket search; a sample of the blocks is also checked
+    against the oracle."""
+    dev = device()
+    mids = torch.from_numpy(onf4.nf4_midpoints()).to(dev)
+    steps = torch.arange(-3, 4, device=dev)
+    m_idx, s_idx, sg = torch.meshgrid(torch.arange(15, device=dev), torch.arange(7, device=dev),
+                                      torch.arange(2, device=dev), indexing="ij")
+    m_idx, s_idx, sg = m_idx.reshape(-1), s_idx.reshape(-1), sg.reshape(-1)          # 210 combinations
+    per_a = 4 * 64                                     # four blocks per absmax: slot 0 of each holds a
+    slots = torch.cat([torch.arange(b * 64 + 1, b * 64 + 64, device=dev) for b in range(4)])[:210]
+    chunk = 1 << 18
+    for a0 in range(0, 1 << 23, chunk):
+        a = ((torch.arange(a0, a0 + chunk, device=dev, dtype=torch.int32) | 0x3F800000).view(torch.float32))
+        x = torch.zeros(chunk, per_a, dtype=torch.float32, device=dev)
+        x[:, 0::64] = a[:, None]
+        v = a[:, None] * mids[m_idx][None, :]
+        for k in range(1, 4):                          # move |step| ulps towards the step's sign
+            up = (steps[s_idx] >= k)[None, :]
+            dn = (steps[s_idx] <= -k)[None, :]
+            v = torch.where(up, torch.nextafter(v, torch.full_like(v, float("inf"))), v)
+            v = torch.where(dn, torch.nextafter(v, torch.full_like(v, float("-inf"))), v)
+        v = torch.where((sg == 1)[None, :], -v, v)
+        x[:, slots] = v
+        flat = x.reshape(-1)
+        n = flat.numel()
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+        e4b.e4b_quantize_nf4(flat, n, codes, absmax)
+        am = flat.view(-1, 64).abs().amax(dim=1)
+        assert torch.equal(absmax.view(torch.int32), am.view(torch.int32))
+        y = flat.view(-1, 64) / am[:, None]
+        want = torch.bucketize(y, mids, right=False).to(torch.uint8).reshape(-1)
+        got = torch.stack([codes >> 4, codes & 15], dim=1).reshape(-1)
+        bad = (got != want).nonzero()
+        assert bad.numel() == 0, f"{bad.numel()} codes differ, first at element {int(bad[0]) + a0 * per_a}"
+        if a0 == 0:                                    # the expected side against the oracle on a sample
+            rc, ra = onf4.quantize_nf4(flat[: 4096 * 64].cpu().numpy())
+            assert np.array_equal(codes[: 4096 * 32].cpu().numpy(), rc)
+            assert np.array_equal(absmax[:4096].cpu().numpy().view(np.uint32), ra.view(np.uint32))
