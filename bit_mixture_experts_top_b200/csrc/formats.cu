@@ -76,60 +76,60 @@ __global__ void __launch_bounds__(256) dequant_mxfp4_kernel(const uint32_t* __re
 // most 1/64 wide, midpoints at least 0.08 apart), so per bucket and sign
 // code = base + (y > mid): positive y counts the midpoints below lo and tests
 // the one in [lo, hi); negative y counts those at or below -hi and tests the
-// one in (-hi, -lo].  |y| < 2^-5 lies between the two midpoints next to zero:
-// code 7.  The host builds and checks the table (nf4_bucket_table).
+// one in (-hi, -lo].  |y| < 2^-5 lies between the two midpoints next to zero,
+// code 7, which is also what bucket 0 gives for either sign (no midpoint in it,
+// seven below it), so small quotients are clamped into bucket 0.  Entry 2j + s
+// holds bucket j for sign s.  The host builds and checks the table
+// (nf4_bucket_table).
 constexpr int kNf4Buckets = 161;
-constexpr uint32_t kNf4BucketBias = 122u << 5;        // exponent of 2^-5, five mantissa bits
+constexpr int kNf4BucketBias = 122 << 5;              // exponent of 2^-5, five mantissa bits
 struct Nf4Buckets {
-  uint2 e[2][kNf4Buckets];                            // [sign][bucket]: {midpoint bits (or +inf), base}
+  uint2 e[2 * kNf4Buckets];                           // {midpoint bits (or +inf), base}
 };
 
 // One half-warp per 64-block: each lane holds 4 consecutive fp32 (16 bytes),
 // the half-warp reduces |x| to absmax, each lane emits 4 codes (2 bytes).
-__device__ __forceinline__ void quantize_quad(const float4 v, int64_t q, uint32_t half_mask,
-                                              const uint2 (*s_tab)[kNf4Buckets], uint16_t* __restrict__ codes,
+// Branch-free: every element takes the same instruction sequence.
+__device__ __forceinline__ void quantize_quad(float4 v, int64_t q, uint32_t half_mask,
+                                              const uint2* __restrict__ s_tab, uint16_t* __restrict__ codes,
                                               float* __restrict__ absmax) {
   float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(half_mask, a, off));
-  uint32_t c[4];
-  const float xv[4] = {v.x, v.y, v.z, v.w};
+  if ((threadIdx.x & 15) == 0) absmax[q >> 4] = a;
   // y = fl32(x / a) by Markstein's FMA correction (P. Markstein, "Computation of
   // elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev.
   // 34(1), 1990): with r = RN(1/a), q = RN(x*r), the residual x - a*q is exact in
   // one FMA and RN(q + residual*r) is the correctly rounded quotient unless it
-  // underflows.  |x| <= a here, and an underflowing quotient lies far below the
-  // smallest decision midpoint, so the code is the same either way.
-  const float r = __frcp_rn(a);
+  // underflows (an underflowing quotient lies far below the smallest decision
+  // midpoint, so the code is the same either way).  A block with a tiny absmax
+  // is first scaled by 2^96 (exact, and it changes no quotient) so that 1/a and
+  // the residuals stay normal; an all-zero block takes r = 0, so all its
+  // quotients are 0 and its codes 7.
+  const float sc = a < 0x1p-60f ? 0x1p96f : 1.0f;
+  a *= sc;
+  const float r = a == 0.0f ? 0.0f : __frcp_rn(a);
+  const float xv[4] = {v.x * sc, v.y * sc, v.z * sc, v.w * sc};
+  uint32_t c[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    if (a == 0.0f) {
-      c[i] = 7u;
-    } else {
-      const float q = xv[i] * r;
-      const float y = fmaf(fmaf(-a, q, xv[i]), r, q);
-      const uint32_t bits = __float_as_uint(y);
-      const int j = static_cast<int>(((bits & 0x7FFFFFFFu) >> 18) - kNf4BucketBias);
-      if (j < 0) {
-        c[i] = 7u;
-      } else {
-        const uint2 t = s_tab[bits >> 31][j];
-        c[i] = t.y + (y > __uint_as_float(t.x) ? 1u : 0u);
-      }
-    }
+    const float qq = xv[i] * r;
+    const float y = fmaf(fmaf(-a, qq, xv[i]), r, qq);
+    const uint32_t bits = __float_as_uint(y);
+    // bucket of |y|; the upper clamp only keeps non-finite input inside the table
+    const int j = min(max(static_cast<int>((bits << 1) >> 19) - kNf4BucketBias, 0), kNf4Buckets - 1);
+    const uint2 t = s_tab[__funnelshift_l(bits, static_cast<uint32_t>(j), 1)];   // 2j + sign
+    c[i] = t.y + (y > __uint_as_float(t.x) ? 1u : 0u);
   }
-  const uint32_t b0 = (c[0] << 4) | c[1];
-  const uint32_t b1 = (c[2] << 4) | c[3];
-  codes[q] = static_cast<uint16_t>(b0 | (b1 << 8));
-  if ((threadIdx.x & 15) == 0) absmax[q >> 4] = a;
+  codes[q] = static_cast<uint16_t>(((c[2] * 16u + c[3]) << 8) | (c[0] * 16u + c[1]));
 }
 
 // Each thread takes two quads per trip (q and q + stride): two loads in flight.
 __global__ void __launch_bounds__(256) quantize_nf4_kernel(const float4* __restrict__ x, int64_t quads,
                                                              uint16_t* __restrict__ codes,
                                                              float* __restrict__ absmax, const Nf4Buckets tab) {
-  __shared__ uint2 s_tab[2][kNf4Buckets];
-  for (int i = threadIdx.x; i < 2 * kNf4Buckets; i += blockDim.x) (&s_tab[0][0])[i] = (&tab.e[0][0])[i];
+  __shared__ uint2 s_tab[2 * kNf4Buckets];
+  for (int i = threadIdx.x; i < 2 * kNf4Buckets; i += blockDim.x) s_tab[i] = tab.e[i];
   __syncthreads();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const uint32_t half_mask = 0xFFFFu << (threadIdx.x & 16u);   // this half-warp only
@@ -262,7 +262,8 @@ cudaError_t launch_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, in
 namespace {
 
 // The bucket table of quantize_quad, from the fp32 midpoints; null if a premise fails
-// (a bucket with two midpoints, or a midpoint within 2^-5 of zero).
+// (a bucket with two midpoints, a midpoint within 2^-5 of zero, or a bucket 0
+// whose code is not 7 for either sign).
 const Nf4Buckets* nf4_bucket_table() {
   static Nf4Buckets tab;
   static bool ok = [] {
@@ -280,11 +281,12 @@ const Nf4Buckets* nf4_bucket_table() {
         if (m[i] > -hi && m[i] <= -lo) { mid_n = m[i]; ++inneg; }
       }
       if (inpos > 1 || inneg > 1) return false;
+      if (j == 0 && (base_p != 7 || base_n != 7 || inpos || inneg)) return false;
       uint32_t bp, bn;
       std::memcpy(&bp, &mid_p, 4);
       std::memcpy(&bn, &mid_n, 4);
-      tab.e[0][j] = make_uint2(bp, base_p);
-      tab.e[1][j] = make_uint2(bn, base_n);
+      tab.e[2 * j] = make_uint2(bp, base_p);
+      tab.e[2 * j + 1] = make_uint2(bn, base_n);
     }
     return true;
   }();

@@ -75,6 +75,8 @@ def test_quantize_nf4_random_scales_bit_exact():
         blocks.append((g.standard_normal(64 * 500) * 2.0 ** p).astype(np.float32))
     blocks.append(np.zeros(64 * 3, np.float32))                                   # all-zero blocks
     blocks.append(g.uniform(-1, 1, 64 * 300).astype(np.float32))
+    for p in (-70, -100, -126, -135, -145):                  # tiny absmax: normal, at and below 2^-126
+        blocks.append((g.standard_normal(64 * 200) * 2.0 ** p).astype(np.float32))
     _assert_quant_equal(np.concatenate(blocks))
 
 
