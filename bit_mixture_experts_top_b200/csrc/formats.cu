@@ -106,10 +106,13 @@ __device__ __forceinline__ void quantize_quad(float4 v, int64_t q, uint32_t half
   // is first scaled by 2^96 (exact, and it changes no quotient) so that 1/a and
   // the residuals stay normal; an all-zero block takes r = 0, so all its
   // quotients are 0 and its codes 7.
-  const float sc = a < 0x1p-60f ? 0x1p96f : 1.0f;
-  a *= sc;
+  float xv[4] = {v.x, v.y, v.z, v.w};
+  if (a < 0x1p-60f) {                      // uniform across the half-warp
+    a *= 0x1p96f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] *= 0x1p96f;
+  }
   const float r = a == 0.0f ? 0.0f : __frcp_rn(a);
-  const float xv[4] = {v.x * sc, v.y * sc, v.z * sc, v.w * sc};
   uint32_t c[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
