@@ -255,7 +255,7 @@ __device__ __forceinline__ float e8m0_f32(uint32_t s) {
 // into registers while the current one is multiplied, and the decoded tiles
 // are double-buffered in shared memory (one barrier per slab).
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
+__global__ void __launch_bounds__(256, 3) dgrad_kernel(const DgParams p) {
   extern __shared__ __align__(16) uint8_t dg_smem[];
   uint16_t (*sW)[kDgK][kPadW] = reinterpret_cast<uint16_t (*)[kDgK][kPadW]>(dg_smem);                 // [2][m][n]
   uint16_t (*sA)[kDgTok][kPad] = reinterpret_cast<uint16_t (*)[kDgTok][kPad]>(dg_smem + 2 * kDgK * kPadW * 2);
@@ -336,31 +336,70 @@ __global__ void __launch_bounds__(256) dgrad_kernel(const DgParams p) {
     __syncthreads();
   }
 
-  // epilogue: acc[nt][h * 2 + i] is row 16wt + g + 8h, column 64wn + 8nt + 2c + i of the tile
+  // epilogue: acc[nt][h * 2 + i] is row 16wt + g + 8h, column 64wn + 8nt + 2c + i of the tile;
+  // a thread's columns come in adjacent pairs (i = 0, 1; N is even), moved as one word
+  if constexpr (MODE == 0) {
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int tr = 16 * wt + g + 8 * h;
+        const int n = n0 + 64 * wn + 8 * nt + 2 * c;
+        if (tr >= rows || n >= p.N) continue;
+        const int64_t gi = (r0 + tr) * 2 * p.I + n;
+        const float2 gg = *reinterpret_cast<const float2*>(p.G + gi);
+        const float2 gu = *reinterpret_cast<const float2*>(p.G + gi + p.I);
+        float dg0, du0, dg1, du1;
+        act_grads(p.ep, gg.x, gu.x, dg0, du0);
+        act_grads(p.ep, gg.y, gu.y, dg1, du1);
+        const float v0 = acc[nt][2 * h], v1 = acc[nt][2 * h + 1];
+        *reinterpret_cast<uint32_t*>(p.dG + gi) = pack_bf16x2(v0 * dg0, v1 * dg1);
+        *reinterpret_cast<uint32_t*>(p.dG + gi + p.I) = pack_bf16x2(v0 * du0, v1 * du1);
+      }
+    }
+  } else {
+    // the LoRA term dxa_r A_e^T: the tile's dxa rows (fp32 [64][16]) and A_e rows of
+    // its columns (bf16 [128][16]) are staged in the now idle tile buffers
+    const int rk = p.lora_rank;
+    float* s_dxa = reinterpret_cast<float*>(dg_smem);
+    uint16_t* s_A = reinterpret_cast<uint16_t*>(dg_smem + kDgTok * 16 * 4);
+    if (rk > 0) {
+      for (int i = tid; i < kDgTok * 16; i += 256) {
+        const int rr = i >> 4, j = i & 15;
+        s_dxa[i] = (rr < rows && j < rk) ? p.dxa[static_cast<int64_t>(r0 + rr) * 16 + j] : 0.0f;
+      }
+      for (int i = tid; i < kDgCols * 16; i += 256) {
+        const int cc = i >> 4, j = i & 15;
+        const int n = n0 + cc;
+        s_A[i] = (n < p.N && j < rk) ? p.lora_A[(static_cast<int64_t>(e) * p.N + n) * rk + j] : uint16_t(0);
+      }
+      __syncthreads();
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int tr = 16 * wt + g + 8 * h;
       if (tr >= rows) continue;
+      float dr[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) dr[j] = rk > 0 ? s_dxa[tr * 16 + j] : 0.0f;
       const int64_t r = r0 + tr;
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int n = n0 + 64 * wn + 8 * nt + 2 * c + i;
-        if (n >= p.N) continue;
-        const float v = acc[nt][2 * h + i];
-        if (MODE == 0) {
-          const int64_t gi = r * 2 * p.I + n;
-          float dg, du;
-          act_grads(p.ep, p.G[gi], p.G[gi + p.I], dg, du);
-          p.dG[gi] = __bfloat16_as_ushort(__float2bfloat16_rn(v * dg));
-          p.dG[gi + p.I] = __bfloat16_as_ushort(__float2bfloat16_rn(v * du));
-        } else {
-          float o = v;
-          if (p.lora_rank > 0) {
-            const uint16_t* ar = p.lora_A + (static_cast<int64_t>(e) * p.N + n) * p.lora_rank;
-            const float* dr = p.dxa + r * 16;
-            for (int j = 0; j < p.lora_rank; ++j) o = fmaf(dr[j], bf16_to_f32(ar[j]), o);
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int cc = 64 * wn + 8 * nt + 2 * c + i;
+          const int n = n0 + cc;
+          if (n >= p.N) continue;
+          float o = acc[nt][2 * h + i];
+          if (rk > 0) {
+            const uint4 a0 = *reinterpret_cast<const uint4*>(s_A + cc * 16);
+            const uint4 a1 = *reinterpret_cast<const uint4*>(s_A + cc * 16 + 8);
+            const uint32_t aw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (j >= rk) break;
+              o = fmaf(dr[j], bf16_to_f32((aw[j >> 1] >> (16 * (j & 1))) & 0xFFFFu), o);
+            }
           }
           p.dX[r * p.N + n] = o;
         }
