@@ -8,7 +8,9 @@
 //   * one warp per token; lane l holds the logits of experts l, l+32, ...
 //     packed into 32-bit keys (order-preserving bf16 bits << 16 | 0xFFFF - id),
 //     so one unsigned max picks the largest logit and, on ties, the lowest id;
-//     k rounds of __reduce_max_sync select the k experts;
+//     each lane sorts its keys once, then k rounds of __reduce_max_sync over the
+//     lanes' largest remaining keys select the k experts (keys are unique, so
+//     exactly one lane owns each pick and steps to its next key);
 //   * gate weights are the fp32 softmax of the k selected logits, or (gating
 //     E4B_GATE_SOFTMAX_ALL) the softmax over all E logits read at the k picks,
 //     not renormalised: the denominator is summed from the keys before the
@@ -58,6 +60,51 @@ __device__ __forceinline__ float row_exp_sum(const uint32_t (&key)[J], float m) 
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
   return s;
+}
+
+__device__ __forceinline__ void cas_desc(uint32_t& a, uint32_t& b) {
+  const uint32_t hi = max(a, b), lo = min(a, b);
+  a = hi;
+  b = lo;
+}
+
+// Sorts J <= 8 keys in descending order (Batcher's odd-even merge networks).
+template <int J>
+__device__ __forceinline__ void sort_desc(uint32_t (&x)[J]) {
+  if constexpr (J == 2) {
+    cas_desc(x[0], x[1]);
+  } else if constexpr (J == 4) {
+    cas_desc(x[0], x[1]); cas_desc(x[2], x[3]);
+    cas_desc(x[0], x[2]); cas_desc(x[1], x[3]);
+    cas_desc(x[1], x[2]);
+  } else if constexpr (J == 8) {
+    cas_desc(x[0], x[1]); cas_desc(x[2], x[3]); cas_desc(x[4], x[5]); cas_desc(x[6], x[7]);
+    cas_desc(x[0], x[2]); cas_desc(x[1], x[3]); cas_desc(x[4], x[6]); cas_desc(x[5], x[7]);
+    cas_desc(x[1], x[2]); cas_desc(x[5], x[6]);
+    cas_desc(x[0], x[4]); cas_desc(x[1], x[5]); cas_desc(x[2], x[6]); cas_desc(x[3], x[7]);
+    cas_desc(x[2], x[4]); cas_desc(x[3], x[5]);
+    cas_desc(x[1], x[2]); cas_desc(x[3], x[4]); cas_desc(x[5], x[6]);
+  }
+}
+
+// One token's top k (one warp, keys already loaded, 0 = no expert): lane r < k
+// returns the r-th largest key, and all_sum the full-softmax denominator when
+// `gating` asks for it (summed before any key is taken).
+template <int J>
+__device__ __forceinline__ uint32_t warp_topk(uint32_t (&key)[J], int k, int gating, int lane, float& all_sum) {
+  sort_desc<J>(key);
+  uint32_t mine = 0;
+  for (int r = 0; r < k; ++r) {
+    const uint32_t best = __reduce_max_sync(kFull, key[0]);
+    if (r == 0 && gating == E4B_GATE_SOFTMAX_ALL) all_sum = row_exp_sum(key, key_logit(best));
+    if (key[0] == best) {                  // the owner steps to its next key
+#pragma unroll
+      for (int j = 0; j + 1 < J; ++j) key[j] = key[j + 1];
+      key[J - 1] = 0u;
+    }
+    if (lane == r) mine = best;
+  }
+  return mine;
 }
 
 // Stable rank: block b's slots [s0, s1) take positions base[b][e] + (# earlier
@@ -116,7 +163,8 @@ __global__ void __launch_bounds__(kThreads) route_rank_kernel(const int32_t* __r
   rank_block<kWarps>(blockIdx.x, topk_ids, T, E, k, block_base, sorted_slot, slot_pos, s_wc);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E,
+template <int J>
+__global__ void __launch_bounds__(kTopkThreads, 1) route_topk_kernel(const uint16_t* __restrict__ logits, int T, int E,
                                                                   int k, int gating, int tokens_per_tile, int nblk,
                                                                   int32_t* __restrict__ topk_ids,
                                                                   float* __restrict__ topk_w, int32_t* block_counts,
@@ -135,36 +183,23 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
 
   // warp w takes tokens t_begin + w + kTopkWarps * q; all their logits are loaded first
   const int t_begin = blockIdx.x * kRouteTokensPerBlock;
-  const int per_lane = (E + 31) >> 5;      // <= 8
-  uint32_t key[kTokPerWarp][kMaxExperts / 32];
+  uint32_t key[kTokPerWarp][J];            // J = ceil(E / 32) keys per lane
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
     const int t = t_begin + warp + kTopkWarps * q;
     const uint16_t* row = logits + static_cast<int64_t>(t) * E;
 #pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
+    for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      key[q][j] = (t < T && j < per_lane && e < E) ? route_key(__ldg(row + e), e) : 0u;   // real keys are never 0
+      key[q][j] = (t < T && e < E) ? route_key(__ldg(row + e), e) : 0u;   // real keys are never 0
     }
   }
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
     const int t = t_begin + warp + kTopkWarps * q;
     if (t >= T) break;
-    uint32_t mine = 0;                     // lane j keeps the j-th pick
     float all_sum = 0.0f;                  // full-softmax denominator (E4B_GATE_SOFTMAX_ALL)
-    for (int r = 0; r < k; ++r) {
-      uint32_t best = 0;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
-      best = __reduce_max_sync(kFull, best);
-      if (r == 0 && gating == E4B_GATE_SOFTMAX_ALL) all_sum = row_exp_sum(key[q], key_logit(best));
-      const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j)
-        if (lane + 32 * j == e) key[q][j] = 0u;
-      if (lane == r) mine = best;
-    }
+    const uint32_t mine = warp_topk(key[q], k, gating, lane, all_sum);   // lane j keeps the j-th pick
     int id = 0;
     float v = 0.0f;
     if (lane < k) {
@@ -260,8 +295,8 @@ __global__ void __launch_bounds__(kTopkThreads) route_topk_kernel(const uint16_t
 // forward starts with a single launch.  Decode batches (T <= 32) take an
 // 8-warp block, whose barriers and shared-memory clears cost a quarter of the
 // 32-warp block's.
-template <int NW>
-__global__ void __launch_bounds__(NW * 32) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
+template <int NW, int J>
+__global__ void __launch_bounds__(NW * 32, 1) route_small_kernel(const uint16_t* __restrict__ logits, int T, int E,
                                                                   int k, int gating, int tokens_per_tile,
                                                                   int32_t* status_words,
                                                                   int32_t* __restrict__ topk_ids,
@@ -283,36 +318,23 @@ __global__ void __launch_bounds__(NW * 32) route_small_kernel(const uint16_t* __
   for (int i = tid; i < kW * kMaxExperts; i += kT) (&s_wc[0][0])[i] = 0;
   __syncthreads();
 
-  const int per_lane = (E + 31) >> 5;
-  uint32_t key[kTokPerWarp][kMaxExperts / 32];
+  uint32_t key[kTokPerWarp][J];            // J = ceil(E / 32) keys per lane
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
     const int t = warp + kW * q;
     const uint16_t* row = logits + static_cast<int64_t>(t) * E;
 #pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
+    for (int j = 0; j < J; ++j) {
       const int e = lane + 32 * j;
-      key[q][j] = (t < T && j < per_lane && e < E) ? route_key(__ldg(row + e), e) : 0u;
+      key[q][j] = (t < T && e < E) ? route_key(__ldg(row + e), e) : 0u;
     }
   }
 #pragma unroll
   for (int q = 0; q < kTokPerWarp; ++q) {
     const int t = warp + kW * q;
     if (t >= T) break;
-    uint32_t mine = 0;
     float all_sum = 0.0f;
-    for (int r = 0; r < k; ++r) {
-      uint32_t best = 0;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) best = max(best, key[q][j]);
-      best = __reduce_max_sync(kFull, best);
-      if (r == 0 && gating == E4B_GATE_SOFTMAX_ALL) all_sum = row_exp_sum(key[q], key_logit(best));
-      const int e = 0xFFFF - static_cast<int>(best & 0xFFFFu);
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j)
-        if (lane + 32 * j == e) key[q][j] = 0u;
-      if (lane == r) mine = best;
-    }
+    const uint32_t mine = warp_topk(key[q], k, gating, lane, all_sum);
     int id = 0;
     float v = 0.0f;
     if (lane < k) {
@@ -528,6 +550,34 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const float* __restri
 
 }  // namespace
 
+namespace {
+
+// The routing launches for J = ceil(E / 32) keys per lane (J in {1, 2, 4, 8}).
+template <int J>
+cudaError_t launch_route_keys(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
+                              int32_t tokens_per_tile, const RouteBuffers& b, int32_t* status_words,
+                              cudaStream_t s) {
+  const int nblk = route_blocks(T);
+  if (nblk == 1) {
+    if (T <= 4 * 8)
+      return launch_pdl(route_small_kernel<8, J>, dim3(1), dim3(8 * 32), 0, s, logits, T, E, k, gating,
+                        tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
+                        b.sorted_slot, b.slot_pos);
+    return launch_pdl(route_small_kernel<kTopkWarps, J>, dim3(1), dim3(kTopkThreads), 0, s, logits, T, E, k,
+                      gating, tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
+                      b.sorted_slot, b.slot_pos);
+  }
+  if (status_words && cudaMemsetAsync(status_words, 0, kStatusBytes, s) != cudaSuccess) return cudaGetLastError();
+  cudaError_t err = launch_pdl(route_topk_kernel<J>, dim3(nblk), dim3(kTopkThreads), 0, s, logits, T, E, k, gating,
+                               tokens_per_tile, nblk, b.topk_ids, b.topk_w, b.block_counts, b.done_counter,
+                               b.expert_offsets, b.chunk_off, b.sorted_slot, b.slot_pos);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(route_rank_kernel, dim3(nblk), dim3(kThreads), 0, s, b.topk_ids, T, E, k,
+                    static_cast<const int32_t*>(b.block_counts), b.sorted_slot, b.slot_pos);
+}
+
+}  // namespace
+
 cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k, int32_t gating,
                          int32_t tokens_per_tile,
                          const RouteBuffers& b, int32_t* status_words, cudaStream_t s) {
@@ -537,23 +587,10 @@ cudaError_t launch_route(const uint16_t* logits, int32_t T, int32_t E, int32_t k
     if (err == cudaSuccess && b.chunk_off) err = cudaMemsetAsync(b.chunk_off, 0, sizeof(int32_t) * (E + 1), s);
     return err;
   }
-  const int nblk = route_blocks(T);
-  if (nblk == 1) {
-    if (T <= 4 * 8)
-      return launch_pdl(route_small_kernel<8>, dim3(1), dim3(8 * 32), 0, s, logits, T, E, k, gating,
-                        tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
-                        b.sorted_slot, b.slot_pos);
-    return launch_pdl(route_small_kernel<kTopkWarps>, dim3(1), dim3(kTopkThreads), 0, s, logits, T, E, k, gating,
-                      tokens_per_tile, status_words, b.topk_ids, b.topk_w, b.expert_offsets, b.chunk_off,
-                      b.sorted_slot, b.slot_pos);
-  }
-  if (status_words && cudaMemsetAsync(status_words, 0, kStatusBytes, s) != cudaSuccess) return cudaGetLastError();
-  cudaError_t err = launch_pdl(route_topk_kernel, dim3(nblk), dim3(kTopkThreads), 0, s, logits, T, E, k, gating,
-                               tokens_per_tile, nblk, b.topk_ids, b.topk_w, b.block_counts, b.done_counter,
-                               b.expert_offsets, b.chunk_off, b.sorted_slot, b.slot_pos);
-  if (err != cudaSuccess || nblk == 1) return err;
-  return launch_pdl(route_rank_kernel, dim3(nblk), dim3(kThreads), 0, s, b.topk_ids, T, E, k,
-                    static_cast<const int32_t*>(b.block_counts), b.sorted_slot, b.slot_pos);
+  if (E <= 32) return launch_route_keys<1>(logits, T, E, k, gating, tokens_per_tile, b, status_words, s);
+  if (E <= 64) return launch_route_keys<2>(logits, T, E, k, gating, tokens_per_tile, b, status_words, s);
+  if (E <= 128) return launch_route_keys<4>(logits, T, E, k, gating, tokens_per_tile, b, status_words, s);
+  return launch_route_keys<8>(logits, T, E, k, gating, tokens_per_tile, b, status_words, s);
 }
 
 cudaError_t launch_gather(const uint16_t* x, int32_t H, int32_t k, int32_t R, const int32_t* sorted_slot,
