@@ -495,13 +495,13 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, int32_t T, const uint16_t* lo
   if (T > 0) {
     if (!logits || !dout || !gu_codes || !gu_scales || !dn_codes || !dn_scales || !dx || !dlogits)
       return E4B_ERR_INVALID_ARG;
-    if (!aligned(dout, 4) || !aligned(dx, 16) || !aligned(dlogits, 4) || !aligned(gu_codes, 16) ||
+    if (!aligned(dout, 8) || !aligned(dx, 16) || !aligned(dlogits, 4) || !aligned(gu_codes, 16) ||
         !aligned(dn_codes, 16))
       return E4B_ERR_INVALID_ARG;
     if (dq ? !(valid_dq(static_cast<const e4b_nf4_dq*>(gu_scales)) && valid_dq(static_cast<const e4b_nf4_dq*>(dn_scales)))
            : !(aligned(gu_scales, 16) && aligned(dn_scales, 16)))
       return E4B_ERR_INVALID_ARG;
-    if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 2) || !aligned(dA, 4) || !aligned(dB, 4)))
+    if (lora && (!aligned(lora_A, 2) || !aligned(lora_B, 16) || !aligned(dA, 4) || !aligned(dB, 4)))
       return E4B_ERR_INVALID_ARG;
   }
   BackwardLaunch b;

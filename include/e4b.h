@@ -323,15 +323,17 @@ e4b_status e4b_moe_forward_train(const e4b_moe_desc* d, int32_t T, const uint16_
  * The clamps of E4B_ACT_CLAMPED_GLU pass the gradient inside their range,
  * ends included.
  *   logits  : [T, E] bf16, the forward's                    (device, read)
- *   dout    : [T, H] bf16 upstream gradient                 (device, read)
+ *   dout    : [T, H] bf16 upstream gradient, 8-byte aligned (device, read)
  *   gu_codes, gu_scales, dn_codes, dn_scales, lora_A, lora_B: the forward's
- *   dx      : [T, H] fp32                                   (device, written)
+ *             (lora_B here 16-byte aligned: its rows are read in 16-byte words)
+ *   dx      : [T, H] fp32, 16-byte aligned                  (device, written)
  *   dlogits : [T, E] fp32                                   (device, written)
  *   dA      : [E, H, r] fp32, dB : [E, r, 2I] fp32, with LoRA, else NULL
  *             (device, written; experts no row is routed to get zeros)
  *   ws      : the workspace e4b_moe_forward_train filled
  * Within the forward's tolerance class: bf16 operands (dY, dG and the decoded
- * weights), fp32 accumulation.
+ * weights), fp32 accumulation.  Misaligned or missing pointers return
+ * E4B_ERR_INVALID_ARG before any launch.
  */
 e4b_status e4b_moe_backward(const e4b_moe_desc* d, int32_t T, const uint16_t* logits,
                             const uint16_t* dout, const uint8_t* gu_codes, const void* gu_scales,

@@ -120,6 +120,12 @@ def test_training_entry_validation(L):
     st = L.e4b_moe_backward(ctypes.byref(d), 64, fake, fake, fake, fake, fake, fake, fake, fake, None, fake,
                             fake, fake, fake, tw, None)
     assert st == e4b.E4B_ERR_INVALID_ARG
+    # alignment the backward's word loads need: dout 8 bytes, lora_B 16 bytes, dx 16 bytes
+    for i, bad in ((1, fake + 4), (7, fake + 2), (8, fake + 8)):     # dout, lora_B, dx
+        a = [fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake]
+        a[i] = bad
+        st = L.e4b_moe_backward(ctypes.byref(d), 64, *a, fake, tw, None)
+        assert st == e4b.E4B_ERR_INVALID_ARG, i
 
 
 def test_expand_absmax_dq_validation(L):
