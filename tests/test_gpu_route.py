@@ -36,7 +36,11 @@ def _check(logits_bits, k, gating="topk"):
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 128, 8), (64, 8, 2), (64, 128, 8), (1000, 32, 4), (300, 256, 8),
-                                   (5, 5, 5), (129, 16, 1), (2048, 128, 8), (4096, 32, 4)])
+                                   (5, 5, 5), (129, 16, 1), (2048, 128, 8), (4096, 32, 4),
+                                   # 1, 2, 4 and 8 keys per lane on both one-block widths and the multi-block
+                                   # path, expert counts that are not multiples of 32
+                                   (20, 64, 6), (100, 48, 4), (300, 60, 4), (100, 100, 8), (16, 200, 8),
+                                   (700, 200, 8), (32, 33, 3)])
 def test_route_matches_oracle(T, E, k):
     _check(synth.normal_bf16((T, E), 1.0, 0, f"route{T}_{E}"), k)
 
@@ -58,7 +62,8 @@ def test_route_all_tokens_one_expert():
     _check(synth.to_bf16_bits(lg), 2)
 
 
-@pytest.mark.parametrize("T,E,k", [(64, 128, 8), (5, 5, 5), (1000, 32, 4), (2048, 128, 8), (300, 256, 8)])
+@pytest.mark.parametrize("T,E,k", [(64, 128, 8), (5, 5, 5), (1000, 32, 4), (2048, 128, 8), (300, 256, 8),
+                                   (40, 48, 6), (100, 200, 8)])
 def test_route_full_softmax_gating(T, E, k):
     # one routing block (T <= 128) and the multi-block path; k = E sums to 1
     _check(synth.normal_bf16((T, E), 2.0, 0, f"groute{T}_{E}"), k, "all")
