@@ -61,7 +61,6 @@ constexpr int WARP_RAW = 0;                  // TMA producer of packed codes
 constexpr int WARP_ACT = 1;                  // TMA producer of activation tiles
 constexpr int WARP_MMA = 2;
 constexpr int WARP_DQ0 = 3;
-constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint64_t kDrainNs = 50000000ull;   // error path: wait at most 50 ms per in-flight stage
 
 // Two placements of the dequantised weight tile (the UMMA A operand):

@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(SK_THREADS, 1)
         const Unit un = decode_unit<TOK>(u, p.n_blocks, p.E, s_chunk, s_off);
         int row_a, row_b;
         unit_rows<MODE>(p, un, row_a, row_b);
-        const int ya = un.e * p.N + row_a, yb = un.e * p.N + row_b;
+        const int ya = un.e * p.N + row_a;
         for (int st = 0; st < nst; ++st) {
           if (!mbar_wait(&empty[slot], ph ^ 1u, wctx, 712)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[slot], STAGE_BYTES);
