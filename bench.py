@@ -671,7 +671,8 @@ def bench_e4b(args, world, rank, local):
                     "touched_experts": touched},
         "e2e": {"value": rep.whole_job_rate(T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-                "path": "layer.HostForward.run: pinned host inputs -> device -> forward -> pinned host output, "
+                "path": "layer.HostForward.run: torch copies the inputs from pinned host tensors to the device, "
+                        "the library's forward runs, torch copies the output back to a pinned host tensor; "
                         "one CUDA graph replay and a synchronize per step"},
         "standalone_kernels": formats,
         "configs": configs,
