@@ -80,6 +80,8 @@ class ClockSampler(threading.Thread):
         super().__init__(daemon=True)
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.stop_evt, self.err = period_s, threading.Event(), None
+        self.first = threading.Event()          # set once the first sample is in (or sampling is impossible)
+        self.switch = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -97,6 +99,7 @@ class ClockSampler(threading.Thread):
 
     def run(self):
         if self.nv is None:
+            self.first.set()
             return
         while not self.stop_evt.is_set():
             try:
@@ -107,11 +110,24 @@ class ClockSampler(threading.Thread):
                         self.reasons.add(name)
             except Exception as e:
                 self.err = str(e)
+            self.first.set()
             time.sleep(self.period)
+
+    def start(self):
+        """Starts sampling and returns once the first sample is in; while it runs the interpreter
+        switches threads every 0.2 ms, so a short timed region (whose host thread only enqueues
+        graph replays and then waits) still gets several samples."""
+        self.switch = sys.getswitchinterval()
+        sys.setswitchinterval(2e-4)
+        super().start()
+        self.first.wait(timeout=1.0)
 
     def summary(self):
         self.stop_evt.set()
         self.join(timeout=2)
+        if self.switch is not None:
+            sys.setswitchinterval(self.switch)
+            self.switch = None
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
                 **({"note": self.err} if self.err else {})}

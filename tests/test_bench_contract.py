@@ -29,3 +29,30 @@ def test_command_line_parses():
     assert r.returncode == 0
     for flag in ("--gpus", "--steps", "--warmup", "--impl", "--only-config", "--no-configs"):
         assert flag in r.stdout
+
+
+def test_clock_sampler_samples_a_short_region(monkeypatch):
+    """A 2.4 ms region whose host thread holds the interpreter, then waits (as a timed region of
+    20 decode steps does) gets several samples; the interpreter's switch interval is restored."""
+    import time
+    import types
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 1
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByIndex = lambda i: object()
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    fake.nvmlDeviceGetClockInfo = lambda h, c: 1900
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 | 0x1
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    before = sys.getswitchinterval()
+    c = bench.ClockSampler(0)
+    c.start()
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < 0.0024:
+        n += 1
+    time.sleep(0.002)
+    rec = c.summary()
+    assert rec["samples"] >= 3 and rec["sm_mhz"] == 1900 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["sw_power_cap"]          # gpu_idle is not reported
+    assert sys.getswitchinterval() == before
