@@ -81,7 +81,7 @@ class ClockSampler(threading.Thread):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self.stop_evt, self.err = period_s, threading.Event(), None
         self.first = threading.Event()          # set once the first sample is in (or sampling is impossible)
-        self.switch = None
+        self.switch, self.pre = None, 0
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -121,6 +121,7 @@ class ClockSampler(threading.Thread):
         sys.setswitchinterval(2e-4)
         super().start()
         self.first.wait(timeout=1.0)
+        self.pre = len(self.samples)            # taken before the region: kept only if nothing follows
 
     def summary(self):
         self.stop_evt.set()
@@ -128,6 +129,8 @@ class ClockSampler(threading.Thread):
         if self.switch is not None:
             sys.setswitchinterval(self.switch)
             self.switch = None
+        if len(self.samples) > self.pre:
+            self.samples = self.samples[self.pre:]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
                 **({"note": self.err} if self.err else {})}
